@@ -1,0 +1,14 @@
+"""Float64 CPU oracle for the SSD (Mamba-2) forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this package.  The CUDA
+library never calls it and shares no code with it.
+
+The oracle is the plain definition of the scalar-times-identity selective SSM
+run as a sequential recurrence ("Transformers are SSMs", paperlayer.ai summary,
+§2.4, §3.4.1 and App. B.2.1), written in C (``ssd_oracle.c``) and driven from
+``oracle.py``.  Every function here is pinned by ``tests/test_oracle_pins.py``;
+none is "parity unpinned".
+"""
+
+from .oracle import build, oracle_forward, oracle_threads  # noqa: F401

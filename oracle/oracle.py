@@ -1,0 +1,115 @@
+"""ctypes driver for the float64 C oracle (``ssd_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
+``oracle_forward`` takes host arrays in any float dtype (the test harness passes
+the values the GPU sees, already rounded to the device dtype), upcasts them to
+float64, and returns float64 ``y`` and ``final_states``.  Documents are given
+either implicitly (``batch`` rows of ``seqlen`` tokens) or by ``cu_seqlens``
+(one packed row), exactly as the CUDA boundary takes them.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssd_oracle.c")
+_LIB = os.path.join(_HERE, "libssd_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``ssd_oracle.c`` into ``libssd_oracle.so`` with gcc + OpenMP."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        f = lib.ssd_oracle_forward
+        f.restype = ctypes.c_int
+        f.argtypes = [
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ]
+        lib.ssd_oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def oracle_threads() -> int:
+    """OpenMP threads the oracle uses by default on this host."""
+    return int(_load().ssd_oracle_max_threads())
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # a torch tensor (CPU); bf16 has no numpy dtype
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def oracle_forward(x, dt, A, B, C, D=None, dt_bias=None, initial_states=None,
+                   cu_seqlens=None, heads=None, nthreads: int = 0):
+    """Run the float64 recurrence.
+
+    Shapes (batch mode):  x [b,L,H,P], dt [b,L,H], B/C [b,L,G,N].
+    Shapes (packed mode, ``cu_seqlens`` given): the same with b == 1, and
+    ``initial_states`` / the returned final states are per document.
+    ``heads``: optional list of head indices; only those heads are computed
+    (the other entries of ``y`` / ``final_states`` are returned as NaN).
+    Returns ``(y [b,L,H,P] f64, final_states [ndocs,H,N,P] f64)``.
+    """
+    x = _f64(x)
+    dt = _f64(dt)
+    A = _f64(A)
+    B = _f64(B)
+    C = _f64(C)
+    D = _f64(D)
+    dt_bias = _f64(dt_bias)
+    init = _f64(initial_states)
+    bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    T = bsz * L
+    if cu_seqlens is None:
+        offsets = np.arange(bsz + 1, dtype=np.int64) * L
+    else:
+        if bsz != 1:
+            raise ValueError("cu_seqlens requires a single packed row (batch == 1)")
+        offsets = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    ndocs = len(offsets) - 1
+    if init is not None and init.shape != (ndocs, H, N, P):
+        raise ValueError(f"initial_states must be {(ndocs, H, N, P)}, got {init.shape}")
+    sel = None
+    if heads is not None:
+        sel = np.ascontiguousarray(np.asarray(heads, dtype=np.int32))
+    y = np.full((T, H, P), np.nan)
+    final = np.full((ndocs, H, N, P), np.nan)
+    rc = _load().ssd_oracle_forward(
+        T, H, P, N, G, ndocs, _ptr(offsets),
+        _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(dt_bias), _ptr(init),
+        _ptr(sel), 0 if sel is None else len(sel), _ptr(y), _ptr(final), int(nthreads),
+    )
+    if rc != 0:
+        raise ValueError("ssd_oracle_forward rejected its arguments")
+    return y.reshape(bsz, L, H, P), final
