@@ -1,0 +1,396 @@
+"""Benchmark of the SSD chunked-scan forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one ssd_forward over the whole workload (every step of the path: the
+cumulative decay, the diagonal blocks, the chunk states, the state passing and
+the outputs), inputs resident in HBM.  Each rank runs the full per-GPU workload
+(weak scaling; ranks share nothing, the work has no data-path collective).
+L2 is flushed (a 512 MiB write) before every timed step, outside the timed
+events.  Times are CUDA events on the launching stream, summed over the K
+steps, max over ranks.  ``--impl reference`` times the float64 oracle on the
+host cores on a bounded sample of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSD chunked-scan fwd Mtokens/s and % of roofline (HBM or tensor pipe)"
+DEFAULT_WORKLOAD = "mamba2_130m_layer_b4_L2048"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def algorithmic(w, ndocs):
+    """Compulsory bytes and causal flops of one forward over workload ``w``."""
+    T, H, P, N, G, Q = w.tokens, w.nheads, w.headdim, w.dstate, w.ngroups, w.chunk_size
+    ein = 2 if w.dtype == "bf16" else 4
+    states = ndocs * H * N * P * 4
+    byts = T * H * P * ein * 2 + T * H * ein + 2 * T * G * N * ein + states + 12 * H
+    if w.init != "zero":
+        byts += states
+    flops_tok_head = Q * P + 4 * N * P + Q * N * G / H + 2 * N * P / Q
+    return byts, T * H * flops_tok_head
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "structured_state_space_chunked_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".h")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, path_name):
+    """dram bytes per launch from a committed ncu summary, if the kernels are unchanged."""
+    fn = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(fn) as f:
+            rec = json.load(f)
+        e = rec[workload][path_name]
+        if e.get("source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"]), e.get("kernel")
+    except Exception:
+        pass
+    return None, None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.mark = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def region(self, t0, t1):
+        self.mark = (t0, t1)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        t0, t1 = self.mark or (0, float("inf"))
+        rows = [l for (t, l) in self.lines if t0 - 0.06 <= t <= t1 + 0.06] or [l for _, l in self.lines]
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            parts = [p.strip() for p in r.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- ranks
+def dist_setup(n):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n:
+        raise SystemExit(f"--gpus {n} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    return rank, world, local, pg
+
+
+def barrier(pg):
+    import torch
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(pg, v):
+    import torch
+    if pg is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_sample_throughput(w, inp, budget_s):
+    """Time the oracle on a subset of heads over every sequence of the workload.
+
+    Returns (Mtokens/s in whole-token units, number of heads, seconds): the
+    oracle computed `k` of the H heads for all tokens, i.e. T * k / H whole tokens.
+    """
+    import oracle
+    cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].cpu().numpy()
+    cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+
+    def run(k):
+        t0 = time.perf_counter()
+        oracle.oracle_forward(cpu["x"], cpu["dt"], cpu["A"], cpu["B"], cpu["C"], cpu["D"],
+                              cpu["dt_bias"], cpu["initial_states"], cu_seqlens=cu,
+                              heads=list(range(k)))
+        return time.perf_counter() - t0
+
+    k = 1
+    t = run(k)
+    if t < 0.5 * budget_s and k < w.nheads:
+        k = int(min(w.nheads, max(1, round(k * budget_s / max(t, 1e-6)))))
+        t = run(k)
+    reps = 1
+    if t < 0.25 * budget_s:  # the whole workload is quick: repeat it
+        reps = int(min(50, max(1, 0.5 * budget_s / max(t, 1e-6))))
+        t = sum(run(k) for _ in range(reps)) / reps
+    return (w.tokens * k / w.nheads) / t / 1e6, k, t
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    import torch
+    from structured_state_space_chunked_b200 import inputs as I
+    from structured_state_space_chunked_b200 import ssd
+
+    w = I.workload(args.workload)
+    rank, world, local, pg = dist_setup(args.gpus)
+    hbm_peak, tc_peak, peak_kind = peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import oracle
+        inp = I.make_inputs(w, device="cpu")
+        budget = max(0.05, min(10.0, 150.0 / (args.steps + args.warmup)))
+        _v, kh, _t = oracle_sample_throughput(w, inp, budget)
+        import oracle as _o
+        cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].numpy()
+
+        def ref_step():
+            _o.oracle_forward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                              inp["dt_bias"], inp["initial_states"], cu_seqlens=cu,
+                              heads=list(range(kh)))
+
+        for _ in range(args.warmup):
+            ref_step()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            ref_step()
+        wall = time.perf_counter() - t0
+        value = (w.tokens * kh / w.nheads) * args.steps / wall / 1e6
+        sample = (f"float64 oracle, heads 0..{kh - 1} of {w.nheads} over all {w.tokens} tokens "
+                  f"per step; whole-token throughput = tokens * {kh} / {w.nheads} / time")
+        line = {
+            "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * wall / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name},
+            "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": oracle.oracle_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
+
+    dev = torch.device("cuda", local)
+    inp = I.make_inputs(w, device=dev)
+    ndocs = inp["cu_seqlens"].numel() - 1 if inp["cu_seqlens"] is not None else w.batch
+    bsz, L = inp["x"].shape[:2]
+    h = ssd.SSD(bsz, L, w.nheads, w.headdim, w.dstate, w.ngroups, w.torch_dtype,
+                max_docs=ndocs if inp["cu_seqlens"] is not None else 0, device=dev)
+    path = {"auto": ssd.SSD_PATH_AUTO, "simt": ssd.SSD_PATH_SIMT, "tc": ssd.SSD_PATH_TC}[args.path]
+    if path != ssd.SSD_PATH_AUTO:
+        h.force_path(path)
+    plan = h.plan(w.chunk_size, ndocs if inp["cu_seqlens"] is not None else 0)
+    path_name = {0: "simt", 1: "tc"}[plan.path if path == ssd.SSD_PATH_AUTO else path]
+    y = torch.empty_like(inp["x"])
+    fin = torch.empty(ndocs, w.nheads, w.dstate, w.headdim, dtype=torch.float32, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        h.forward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["dt_bias"],
+                  w.chunk_size, inp["initial_states"], inp["cu_seqlens"], y=y, final_states=fin)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if h.status() != 0:
+        raise SystemExit("device status error during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.2)
+    barrier(pg)
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    barrier(pg)
+    t_wall1 = time.time()
+    clk.region(t_wall0, t_wall1)
+    time.sleep(0.1)
+    clocks = clk.stop()
+    st = h.status()
+    if st != 0:
+        raise SystemExit(f"device status {st} in the timed region")
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    ms = max_over_ranks(pg, ms)
+    tokens_all = w.tokens * world
+    value = tokens_all / (ms * 1e-3) / 1e6
+
+    byts, flops = algorithmic(w, ndocs)
+    achieved_gbs = byts / (ms * 1e-3) / 1e9
+    achieved_tf = flops / (ms * 1e-3) / 1e12
+    traffic, traffic_kernel = recorded_traffic(w.name, path_name)
+    t_hbm = byts / (hbm_peak * 1e9)
+    t_tc = flops / (tc_peak * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved_gbs / hbm_peak, "traffic": traffic}
+    else:
+        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved_tf / tc_peak, "traffic": traffic}
+    roof.update({"peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == "measured"
+                 else "fallback", "algorithmic_bytes_per_launch": byts,
+                 "causal_flops_per_launch": flops, "tensor_tflops_achieved": achieved_tf,
+                 "roofline_us": 1e6 * max(t_hbm, t_tc), "frac_of_roofline": 1e3 * max(t_hbm, t_tc) / ms,
+                 "kernel": traffic_kernel or ("ssd_tc_fused" if path_name == "tc" else "simt (4-5 kernels)")})
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in inp.items()}
+    yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    fh = torch.empty(fin.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for k, v in host.items() if v is not None)
+    d2h = yh.numel() * yh.element_size() + fh.numel() * fh.element_size()
+
+    def e2e_step():
+        h.forward_host(host["x"], host["dt"], host["A"], host["B"], host["C"], host["D"],
+                       host["dt_bias"], w.chunk_size, host["initial_states"], host["cu_seqlens"],
+                       y=yh, final_states=fh)
+
+    for _ in range(3):
+        e2e_step()
+    barrier(pg)
+    t0 = time.perf_counter()
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    barrier(pg)
+    e2e_s = max_over_ranks(pg, (time.perf_counter() - t0) / args.e2e_steps)
+    e2e = {"value": tokens_all / e2e_s / 1e6, "unit": "Mtokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * e2e_s}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        v, kh, t = oracle_sample_throughput(w, inp, 12.0)
+        cpu = {"value": v, "unit": "Mtokens/s", "cores": oracle.oracle_threads(), "kind": "oracle",
+               "sample": f"float64 oracle, heads 0..{kh - 1} of {w.nheads} over all {w.tokens} "
+                         f"tokens in {t:.2f} s; whole-token throughput = tokens * {kh} / "
+                         f"{w.nheads} / time"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                       "nheads": w.nheads, "headdim": w.headdim, "dstate": w.dstate,
+                       "ngroups": w.ngroups, "chunk_size": w.chunk_size,
+                       "tokens_per_gpu": w.tokens, "path": path_name,
+                       "parallelism": f"dp{world} (independent replicas)",
+                       "l2": "flushed before every timed step (512 MiB write, outside the events)"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(plan.kernels) * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    h.close()
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,208 @@
+/*
+ * ssd.h -- C ABI of libssd_b200: the forward pass of the chunked SSD scan
+ * (the state-space-duality layer of Mamba-2) on NVIDIA B200 (sm_100a).
+ *
+ * What is computed ("Transformers are SSMs: Generalized Models and Efficient
+ * Algorithms Through Structured State Space Duality", paperlayer.ai summary):
+ * the selective SSM with scalar-times-identity transitions (§2.4), per head h
+ * and token t of a document, with g = h / (H/G) the B/C group of the head
+ * (shared B, C across heads, §7.1-§7.2):
+ *
+ *     delta_t = softplus(dt[t,h] + dt_bias[h])
+ *     S_t     = exp(delta_t A[h]) S_{t-1} + delta_t B[t,g,:]^T x[t,h,:]      (N x P)
+ *     y[t,h]  = C[t,g,:] S_t + D[h] x[t,h,:]
+ *
+ * with S_{start-1} the document's initial state, evaluated by the block
+ * decomposition of §6: quadratic (masked attention) form on the diagonal
+ * blocks (§6.1), chunk states from the right factors, a scalar scan of states
+ * across chunks and outputs from the left factors (§6.2).  Documents never
+ * exchange information (§8.3 Variable Length); the final state of each
+ * document is returned so that a later call can continue from it (§8.2
+ * Sequence Parallelism: each worker starts from an initial state and passes
+ * its final state on).
+ *
+ * Conventions for every entry point:
+ *  - Return value: SSD_OK (0) or a negative SSD_ERR_* code.  No C++ exception
+ *    crosses this boundary.  ssd_error_string() names a code.
+ *  - Device pointers are CUDA global-memory pointers on the handle's device,
+ *    contiguous, row-major (last index fastest), 16-byte aligned.  The caller
+ *    owns every buffer it passes; the library only reads inputs and writes
+ *    outputs during the work it enqueues.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and is asynchronous: ssd_forward never synchronises.  Buffers
+ *    must stay valid until that work completes.
+ *  - A handle is not thread-safe: concurrent ssd_forward calls on one handle
+ *    share its workspace and race.  Use one handle per stream.
+ *  - Device-side failures (an invalid cu_seqlens array, a bounded wait that
+ *    gave up) are recorded in a status word read by ssd_get_status().
+ */
+#ifndef SSD_B200_H
+#define SSD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+typedef struct CUstream_st* ssd_stream_t; /* same type as cudaStream_t */
+
+/* element types */
+enum { SSD_F32 = 0, SSD_BF16 = 1 };
+
+/* return codes */
+enum {
+  SSD_OK = 0,
+  SSD_ERR_INVALID_ARG = -1, /* null required pointer, bad size, misaligned pointer */
+  SSD_ERR_UNSUPPORTED = -2, /* shape or dtype outside what the library implements */
+  SSD_ERR_CUDA = -3,        /* a CUDA runtime call or kernel launch failed */
+  SSD_ERR_TIMEOUT = -4,     /* a device-side bounded wait gave up (status word) */
+  SSD_ERR_OOM = -5,         /* device allocation failed */
+  SSD_ERR_BAD_SEQLENS = -6  /* cu_seqlens not 0 = c[0] <= ... <= c[n] = tokens (status word) */
+};
+
+/* kernel paths (ssd_plan_t.path, SSD_OPT_FORCE_PATH) */
+enum {
+  SSD_PATH_AUTO = -1,
+  SSD_PATH_SIMT = 0, /* chunk-parallel CUDA-core kernels, fp32 arithmetic (any shape, f32 or bf16) */
+  SSD_PATH_TC = 1    /* fused persistent tcgen05/TMEM kernel (bf16 inputs, fp32 accumulate) */
+};
+
+/* handle options (ssd_set_option) */
+enum {
+  SSD_OPT_FORCE_PATH = 1 /* value: SSD_PATH_AUTO (default), SSD_PATH_SIMT or SSD_PATH_TC */
+};
+
+/*
+ * Problem description, fixed for the life of a handle.
+ *   batch, seqlen   sequences of `seqlen` tokens each; tokens = batch * seqlen.
+ *   nheads H, headdim P, dstate N, ngroups G (H % G == 0; head h reads group
+ *                   h / (H/G)).  Typical head dimensions are 64 and 128 (§2.4).
+ *   in_dtype        SSD_F32 or SSD_BF16: the type of x, dt, B and C.
+ *   out_dtype       SSD_F32 or SSD_BF16: the type of y.
+ *   max_docs        0: sequences are the batch rows.  > 0: ssd_forward may be
+ *                   given cu_seqlens with up to max_docs documents packed into
+ *                   one row (then batch must be 1; §8.3 padding-free packing).
+ *   flags           reserved, must be 0.
+ */
+typedef struct {
+  int64_t batch;
+  int64_t seqlen;
+  int32_t nheads;
+  int32_t headdim;
+  int32_t dstate;
+  int32_t ngroups;
+  int32_t in_dtype;
+  int32_t out_dtype;
+  int32_t max_docs;
+  int32_t flags;
+} ssd_desc_t;
+
+typedef struct ssd_handle_s* ssd_handle_t;
+
+/* What ssd_forward would run for a given call (host-only query, no GPU needed). */
+typedef struct {
+  int32_t path;            /* SSD_PATH_SIMT or SSD_PATH_TC */
+  int32_t num_docs;        /* documents of the call */
+  int64_t num_chunks_max;  /* upper bound on chunks (SIMT path) */
+  int64_t workspace_bytes; /* device workspace the call needs */
+  int32_t units;           /* work units of the TC path (document x head x P-slice), else 0 */
+  int32_t kernels;         /* kernel launches one ssd_forward call makes */
+} ssd_plan_t;
+
+/*
+ * ssd_validate_desc: checks a description without touching the GPU.
+ * Returns SSD_OK, SSD_ERR_INVALID_ARG (non-positive sizes, bad dtype, flags != 0,
+ * max_docs > 0 with batch != 1) or SSD_ERR_UNSUPPORTED (H % G != 0,
+ * P or N outside [1, 256]).
+ */
+SSD_API int ssd_validate_desc(const ssd_desc_t* desc);
+
+/*
+ * ssd_plan: the kernel path and workspace a call with this chunk size and
+ * document count would use (num_docs = 0 for batch mode).  Host only.
+ * chunk_size must be in [1, 256] (the chunk length Q of §6).
+ */
+SSD_API int ssd_plan(const ssd_desc_t* desc, int chunk_size, int num_docs, ssd_plan_t* out);
+
+/*
+ * ssd_create: validates `desc`, selects the current CUDA device, allocates a
+ * small device status word and returns a handle in *out.  Workspace for the
+ * chunk-parallel path is allocated on first use by ssd_forward, stream-ordered
+ * (cudaMallocAsync on the call's stream), and grown when a later call needs
+ * more.  Errors: those of ssd_validate_desc, SSD_ERR_CUDA, SSD_ERR_OOM.
+ */
+SSD_API int ssd_create(const ssd_desc_t* desc, ssd_handle_t* out);
+
+/* ssd_set_option: see SSD_OPT_*.  SSD_ERR_INVALID_ARG for an unknown option or value. */
+SSD_API int ssd_set_option(ssd_handle_t h, int option, int value);
+
+/*
+ * ssd_forward: y, final_states = SSD(x, dt, A, B, C, D, dt_bias, initial_states).
+ *
+ *   x        [batch, seqlen, H, P]  in_dtype     (device)
+ *   dt       [batch, seqlen, H]     in_dtype     (device) raw step before softplus
+ *   A        [H] float32, negative               (device) scalar-times-identity A (§2.4)
+ *   B, C     [batch, seqlen, G, N]  in_dtype     (device)
+ *   D        [H] float32 or NULL (no skip term)  (device)
+ *   dt_bias  [H] float32 or NULL (zero bias)     (device)
+ *   chunk_size  Q in [1, 256]: the chunk length of the block decomposition.
+ *               The result does not depend on Q except through rounding.
+ *   initial_states  [ndocs, H, N, P] float32 or NULL (zero)  (device)
+ *   cu_seqlens  NULL (documents = batch rows, ndocs = batch) or int32
+ *               [num_docs + 1] on the device with 0 = c[0] <= c[1] <= ... <=
+ *               c[num_docs] = batch*seqlen (empty documents allowed); needs
+ *               batch == 1 and 1 <= num_docs <= max_docs.  A violation found on
+ *               the device sets SSD_ERR_BAD_SEQLENS in the status word and the
+ *               call then writes no output.
+ *   num_docs    documents in cu_seqlens (ignored when cu_seqlens is NULL).
+ *   y        [batch, seqlen, H, P] out_dtype (device, written)
+ *   final_states [ndocs, H, N, P] float32 or NULL (device, written): the state
+ *               after each document's last token (its initial state if empty).
+ * Errors (before anything is enqueued): SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED
+ * (a forced path that cannot run this shape), SSD_ERR_OOM; SSD_ERR_CUDA if a
+ * launch fails.
+ */
+SSD_API int ssd_forward(ssd_handle_t h, const void* x, const void* dt, const float* A,
+                const void* B, const void* C, const float* D, const float* dt_bias,
+                int chunk_size, const float* initial_states, const int32_t* cu_seqlens,
+                int num_docs, void* y, float* final_states, ssd_stream_t stream);
+
+/*
+ * ssd_forward_host: the same computation with every array in HOST memory
+ * (pageable or pinned; cu_seqlens too, then num_docs is read from the caller).
+ * Copies the inputs to handle-owned device buffers on `stream`, runs
+ * ssd_forward, copies y and final_states back, and synchronises `stream`
+ * before returning.  The device buffers are allocated on first use and kept.
+ */
+SSD_API int ssd_forward_host(ssd_handle_t h, const void* x, const void* dt, const float* A,
+                     const void* B, const void* C, const float* D, const float* dt_bias,
+                     int chunk_size, const float* initial_states, const int32_t* cu_seqlens,
+                     int num_docs, void* y, float* final_states, ssd_stream_t stream);
+
+/*
+ * ssd_get_status: synchronises `stream`, returns the first device-side error
+ * recorded since the last call (SSD_OK if none) and clears it.
+ */
+SSD_API int ssd_get_status(ssd_handle_t h, ssd_stream_t stream);
+
+/* ssd_destroy: synchronises the device and frees everything the handle owns. NULL is a no-op. */
+SSD_API int ssd_destroy(ssd_handle_t h);
+
+/* Static string naming a return code. */
+SSD_API const char* ssd_error_string(int code);
+
+/* Library version string. */
+SSD_API const char* ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSD_B200_H */

@@ -1,0 +1,332 @@
+// ssd_api.cu -- the C ABI declared in include/ssd.h: argument checks, path
+// selection, workspace management and launches.  All compute runs in the
+// kernels of ssd_simt.cu and ssd_tc.cu.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "ssd_internal.h"
+
+struct ssd_handle_s {
+  ssd_desc_t desc;
+  int device;
+  int num_sms;
+  int force_path;
+  int* status;          // device status word (first error code, 0 = ok)
+  void* ws;             // stream-ordered workspace
+  size_t ws_bytes;
+  void* io;             // device buffers of ssd_forward_host
+  size_t io_bytes;
+};
+
+namespace {
+
+using ssd::Geom;
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+size_t elem_bytes(int dt) { return dt == SSD_BF16 ? 2 : 4; }
+
+int make_geom(const ssd_desc_t& d, int chunk_size, bool varlen, int num_docs, Geom* g) {
+  g->tokens = d.batch * d.seqlen;
+  g->seqlen = d.seqlen;
+  g->H = d.nheads;
+  g->P = d.headdim;
+  g->N = d.dstate;
+  g->G = d.ngroups;
+  g->Q = chunk_size;
+  g->varlen = varlen ? 1 : 0;
+  g->ndocs = varlen ? num_docs : (int)d.batch;
+  if (varlen)
+    g->nchunks_max = (g->tokens + chunk_size - 1) / chunk_size + num_docs;
+  else
+    g->nchunks_max = d.batch * ((d.seqlen + chunk_size - 1) / chunk_size);
+  g->in_bf16 = d.in_dtype == SSD_BF16;
+  g->out_bf16 = d.out_dtype == SSD_BF16;
+  return SSD_OK;
+}
+
+int check_call(const ssd_desc_t& d, int chunk_size, const int32_t* cu, int num_docs) {
+  if (chunk_size < 1 || chunk_size > 256) return SSD_ERR_INVALID_ARG;
+  if (cu) {
+    if (d.max_docs <= 0 || d.batch != 1) return SSD_ERR_INVALID_ARG;
+    if (num_docs < 1 || num_docs > d.max_docs) return SSD_ERR_INVALID_ARG;
+  }
+  return SSD_OK;
+}
+
+int choose_path(const ssd_desc_t& d, const Geom& g, int force) {
+  const bool tc = ssd::tc_supported(g, nullptr);
+  if (force == SSD_PATH_SIMT) return SSD_PATH_SIMT;
+  if (force == SSD_PATH_TC) return tc ? SSD_PATH_TC : SSD_ERR_UNSUPPORTED;
+  (void)d;
+  return tc ? SSD_PATH_TC : SSD_PATH_SIMT;
+}
+
+size_t workspace_for(const Geom& g, int path) {
+  return path == SSD_PATH_TC ? ssd::tc_workspace_bytes(g) : ssd::simt_workspace_bytes(g);
+}
+
+int cuda_rc(cudaError_t e) {
+  if (e == cudaSuccess) return SSD_OK;
+  if (e == cudaErrorMemoryAllocation) return SSD_ERR_OOM;
+  return SSD_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssd_validate_desc(const ssd_desc_t* d) {
+  if (!d) return SSD_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->seqlen < 0 || d->nheads <= 0 || d->headdim <= 0 || d->dstate <= 0 ||
+      d->ngroups <= 0)
+    return SSD_ERR_INVALID_ARG;
+  if (d->in_dtype != SSD_F32 && d->in_dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+  if (d->out_dtype != SSD_F32 && d->out_dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+  if (d->flags != 0 || d->max_docs < 0) return SSD_ERR_INVALID_ARG;
+  if (d->max_docs > 0 && d->batch != 1) return SSD_ERR_INVALID_ARG;
+  if (d->batch * d->seqlen > ((int64_t)1 << 40)) return SSD_ERR_UNSUPPORTED;
+  if (d->nheads % d->ngroups != 0) return SSD_ERR_UNSUPPORTED;
+  if (d->headdim > 256 || d->dstate > 256) return SSD_ERR_UNSUPPORTED;
+  return SSD_OK;
+}
+
+int ssd_plan(const ssd_desc_t* desc, int chunk_size, int num_docs, ssd_plan_t* out) {
+  int rc = ssd_validate_desc(desc);
+  if (rc) return rc;
+  if (!out) return SSD_ERR_INVALID_ARG;
+  const bool varlen = num_docs > 0;
+  rc = check_call(*desc, chunk_size, varlen ? (const int32_t*)1 : nullptr, num_docs);
+  if (rc) return rc;
+  Geom g;
+  make_geom(*desc, chunk_size, varlen, num_docs, &g);
+  const int path = choose_path(*desc, g, SSD_PATH_AUTO);
+  memset(out, 0, sizeof(*out));
+  out->path = path;
+  out->num_docs = g.ndocs;
+  out->num_chunks_max = g.nchunks_max;
+  out->workspace_bytes = (int64_t)workspace_for(g, path);
+  out->units = path == SSD_PATH_TC ? ssd::tc_units(g) : 0;
+  out->kernels = path == SSD_PATH_TC ? ssd::tc_kernels(g) : ssd::simt_kernels(g);
+  return SSD_OK;
+}
+
+int ssd_create(const ssd_desc_t* desc, ssd_handle_t* out) {
+  int rc = ssd_validate_desc(desc);
+  if (rc) return rc;
+  if (!out) return SSD_ERR_INVALID_ARG;
+  *out = nullptr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return SSD_ERR_CUDA;
+  ssd_handle_s* h = new (std::nothrow) ssd_handle_s();
+  if (!h) return SSD_ERR_OOM;
+  h->desc = *desc;
+  h->device = dev;
+  h->num_sms = sms;
+  h->force_path = SSD_PATH_AUTO;
+  cudaError_t e = cudaMalloc(&h->status, sizeof(int) * 4);
+  if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int) * 4);
+  if (e != cudaSuccess) {
+    if (h->status) cudaFree(h->status);
+    delete h;
+    return cuda_rc(e);
+  }
+  *out = h;
+  return SSD_OK;
+}
+
+int ssd_set_option(ssd_handle_t h, int option, int value) {
+  if (!h) return SSD_ERR_INVALID_ARG;
+  if (option == SSD_OPT_FORCE_PATH) {
+    if (value != SSD_PATH_AUTO && value != SSD_PATH_SIMT && value != SSD_PATH_TC)
+      return SSD_ERR_INVALID_ARG;
+    h->force_path = value;
+    return SSD_OK;
+  }
+  return SSD_ERR_INVALID_ARG;
+}
+
+int ssd_forward(ssd_handle_t h, const void* x, const void* dt, const float* A, const void* B,
+                const void* C, const float* D, const float* dt_bias, int chunk_size,
+                const float* initial_states, const int32_t* cu_seqlens, int num_docs, void* y,
+                float* final_states, ssd_stream_t stream_) {
+  if (!h) return SSD_ERR_INVALID_ARG;
+  const ssd_desc_t& d = h->desc;
+  int rc = check_call(d, chunk_size, cu_seqlens, num_docs);
+  if (rc) return rc;
+  const int64_t tokens = d.batch * d.seqlen;
+  if (tokens > 0 && (!x || !dt || !B || !C || !y)) return SSD_ERR_INVALID_ARG;
+  if (!A) return SSD_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) ||
+      !aligned(dt, elem_bytes(d.in_dtype)) || !aligned(A, 4) || !aligned(D, 4) ||
+      !aligned(dt_bias, 4) || !aligned(initial_states, 16) || !aligned(final_states, 16) ||
+      !aligned(cu_seqlens, 4))
+    return SSD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  Geom g;
+  make_geom(d, chunk_size, cu_seqlens != nullptr, num_docs, &g);
+  const int path = choose_path(d, g, h->force_path);
+  if (path < 0) return path;
+
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return SSD_ERR_CUDA;
+
+  const size_t need = workspace_for(g, path);
+  if (need > h->ws_bytes) {
+    if (h->ws) cudaFreeAsync(h->ws, stream);
+    h->ws = nullptr;
+    h->ws_bytes = 0;
+    cudaError_t e = cudaMallocAsync(&h->ws, need, stream);
+    if (e != cudaSuccess) {
+      h->ws = nullptr;
+      if (cur != h->device) cudaSetDevice(cur);
+      return cuda_rc(e);
+    }
+    h->ws_bytes = need;
+  }
+  ssd::Args a{x, dt, A, B, C, D, dt_bias, initial_states, cu_seqlens, y, final_states};
+  cudaError_t e;
+  if (path == SSD_PATH_TC) {
+    e = ssd::tc_forward(g, a, h->ws, h->status, stream, h->num_sms);
+  } else {
+    ssd::SimtWorkspace ws;
+    ssd::simt_carve_workspace(g, h->ws, &ws);
+    e = ssd::simt_forward(g, a, ws, h->status, stream);
+  }
+  if (cur != h->device) cudaSetDevice(cur);
+  return cuda_rc(e);
+}
+
+int ssd_forward_host(ssd_handle_t h, const void* x, const void* dt, const float* A,
+                     const void* B, const void* C, const float* D, const float* dt_bias,
+                     int chunk_size, const float* initial_states, const int32_t* cu_seqlens,
+                     int num_docs, void* y, float* final_states, ssd_stream_t stream_) {
+  if (!h) return SSD_ERR_INVALID_ARG;
+  const ssd_desc_t& d = h->desc;
+  int rc = check_call(d, chunk_size, cu_seqlens, num_docs);
+  if (rc) return rc;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const int64_t T = d.batch * d.seqlen;
+  const int ndocs = cu_seqlens ? num_docs : (int)d.batch;
+  const int maxdocs = d.max_docs > 0 ? d.max_docs : (int)d.batch;
+  const size_t ein = elem_bytes(d.in_dtype), eout = elem_bytes(d.out_dtype);
+  const size_t bx = (size_t)T * d.nheads * d.headdim * ein;
+  const size_t bdt = (size_t)T * d.nheads * ein;
+  const size_t bbc = (size_t)T * d.ngroups * d.dstate * ein;
+  const size_t bh = sizeof(float) * d.nheads;
+  const size_t by = (size_t)T * d.nheads * d.headdim * eout;
+  const size_t bst = sizeof(float) * (size_t)maxdocs * d.nheads * d.dstate * d.headdim;
+  const size_t bcu = sizeof(int32_t) * ((size_t)maxdocs + 1);
+  auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  const size_t off_x = 0, off_dt = off_x + up(bx), off_B = off_dt + up(bdt),
+               off_C = off_B + up(bbc), off_A = off_C + up(bbc), off_D = off_A + up(bh),
+               off_bias = off_D + up(bh), off_init = off_bias + up(bh), off_fin = off_init + up(bst),
+               off_cu = off_fin + up(bst), off_y = off_cu + up(bcu), total = off_y + up(by);
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return SSD_ERR_CUDA;
+  if (h->io_bytes < total) {
+    if (h->io) cudaFree(h->io);
+    h->io = nullptr;
+    h->io_bytes = 0;
+    cudaError_t e = cudaMalloc(&h->io, total);
+    if (e != cudaSuccess) {
+      h->io = nullptr;
+      if (cur != h->device) cudaSetDevice(cur);
+      return cuda_rc(e);
+    }
+    h->io_bytes = total;
+  }
+  char* base = static_cast<char*>(h->io);
+  const size_t bst_call = sizeof(float) * (size_t)ndocs * d.nheads * d.dstate * d.headdim;
+  cudaError_t e = cudaSuccess;
+  auto h2d = [&](size_t off, const void* src, size_t n) {
+    if (src && n && e == cudaSuccess)
+      e = cudaMemcpyAsync(base + off, src, n, cudaMemcpyHostToDevice, stream);
+  };
+  h2d(off_x, x, bx);
+  h2d(off_dt, dt, bdt);
+  h2d(off_B, B, bbc);
+  h2d(off_C, C, bbc);
+  h2d(off_A, A, bh);
+  h2d(off_D, D, bh);
+  h2d(off_bias, dt_bias, bh);
+  h2d(off_init, initial_states, bst_call);
+  h2d(off_cu, cu_seqlens, cu_seqlens ? sizeof(int32_t) * ((size_t)num_docs + 1) : 0);
+  if (e != cudaSuccess) {
+    if (cur != h->device) cudaSetDevice(cur);
+    return cuda_rc(e);
+  }
+  rc = ssd_forward(h, base + off_x, base + off_dt, (const float*)(base + off_A), base + off_B,
+                   base + off_C, D ? (const float*)(base + off_D) : nullptr,
+                   dt_bias ? (const float*)(base + off_bias) : nullptr, chunk_size,
+                   initial_states ? (const float*)(base + off_init) : nullptr,
+                   cu_seqlens ? (const int32_t*)(base + off_cu) : nullptr, num_docs, base + off_y,
+                   final_states ? (float*)(base + off_fin) : nullptr, stream_);
+  if (rc == SSD_OK) {
+    if (y) e = cudaMemcpyAsync(y, base + off_y, by, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess && final_states)
+      e = cudaMemcpyAsync(final_states, base + off_fin, bst_call, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    rc = cuda_rc(e);
+  }
+  if (cur != h->device) cudaSetDevice(cur);
+  return rc;
+}
+
+int ssd_get_status(ssd_handle_t h, ssd_stream_t stream_) {
+  if (!h) return SSD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return SSD_ERR_CUDA;
+  int v = 0;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess) e = cudaMemcpy(&v, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && v != 0) e = cudaMemset(h->status, 0, sizeof(int));
+  if (cur != h->device) cudaSetDevice(cur);
+  if (e != cudaSuccess) return SSD_ERR_CUDA;
+  return v;
+}
+
+int ssd_destroy(ssd_handle_t h) {
+  if (!h) return SSD_OK;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cur != h->device) cudaSetDevice(h->device);
+  cudaError_t e = cudaDeviceSynchronize();
+  if (h->ws) {
+    cudaFreeAsync(h->ws, 0);
+    cudaStreamSynchronize(0);
+  }
+  if (h->io) cudaFree(h->io);
+  if (h->status) cudaFree(h->status);
+  if (cur != h->device) cudaSetDevice(cur);
+  delete h;
+  return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+const char* ssd_error_string(int code) {
+  switch (code) {
+    case SSD_OK: return "SSD_OK";
+    case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG: invalid argument";
+    case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: shape or dtype not supported";
+    case SSD_ERR_CUDA: return "SSD_ERR_CUDA: CUDA runtime error";
+    case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: a device-side wait gave up";
+    case SSD_ERR_OOM: return "SSD_ERR_OOM: device allocation failed";
+    case SSD_ERR_BAD_SEQLENS: return "SSD_ERR_BAD_SEQLENS: cu_seqlens is not a valid partition";
+    default: return "SSD_ERR_UNKNOWN";
+  }
+}
+
+const char* ssd_version(void) { return "ssd_b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

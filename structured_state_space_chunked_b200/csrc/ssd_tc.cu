@@ -1,0 +1,803 @@
+// ssd_tc.cu -- fused SSD forward on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One persistent kernel.  A work unit is (document, head, 64-wide slice of the
+// head dimension P); a CTA walks the unit's tokens in tiles of 128 and keeps the
+// running SSM state of the slice in tensor memory the whole way, so chunk states
+// never touch HBM.  Per tile j (tokens t0..t0+127 of one document):
+//
+//   cs_l   = sum_{k<=l} delta_k A            (in-tile cumulative log decay, §3.2.2)
+//   Z      = C_j B_j^T                       (128 x 128, tensor cores)
+//   M[l,s] = Z[l,s] exp(cs_l - cs_s) delta_s for s <= l, 0 above; M[l,l] += D
+//                                            (the masked quadratic form of the
+//                                             diagonal block, §6.1 / §5.1)
+//   Ydiag  = M x_j                           (tensor cores)
+//   Yoff   = C_j H_j                         (left factors, §6.2; H_j = state
+//                                             entering the tile, bf16 copy)
+//   y      = exp(cs_l) Yoff + Ydiag
+//   H_{j+1}= exp(cs_127) H_j + B_j^T (w o x_j),  w_s = exp(cs_127 - cs_s) delta_s
+//                                            (right factors + the scalar scan
+//                                             across chunks, §6.2), accumulated
+//                                             by the tensor cores onto the
+//                                             decayed state in TMEM.
+//
+// A chunk of Q = 128 or 256 tokens ("Transformers are SSMs", paperlayer.ai
+// summary, §6) is processed as Q/128 such tiles: for Q = 256 the strictly lower
+// 128 x 128 block of the chunk's quadratic form goes through the same rank-N
+// factorisation the decomposition uses between chunks (the mask L restricted to
+// a strictly lower block is rank one, §3.2.2), which equals the quadratic form
+// up to rounding.
+//
+// Roles: warp 0 issues TMA loads (double-buffered x/B/C tiles), warp 1 owns TMEM
+// and one thread issues every tcgen05.mma, warps 2..5 are the epilogue
+// (cumsum, decay mask, state rescale, outputs).  Every mbarrier wait is bounded:
+// on expiry the CTA records SSD_ERR_TIMEOUT in the status word and unwinds.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssd_internal.h"
+
+namespace ssd {
+namespace {
+
+constexpr int kTile = 128;     // tokens per tile
+constexpr int kPT = 64;        // head-dim columns per unit
+constexpr int kThreads = 192;  // 6 warps
+constexpr uint32_t kPanel = 16384;  // one 128-row x 128-byte SW128 panel
+
+template <int NT>
+struct Cfg {
+  static constexpr int NPAD = 128 * NT;        // state dim padded to the lane tiles
+  static constexpr int NPANEL = 2 * NT;        // 64-column panels of a B/C tile
+  static constexpr int NSTAGE = NT == 1 ? 2 : 1;
+  static constexpr uint32_t X_BYTES = kPanel;
+  static constexpr uint32_t BC_BYTES = NPANEL * kPanel;
+  static constexpr uint32_t STAGE_BYTES = X_BYTES + 2 * BC_BYTES;
+  static constexpr uint32_t OFF_M = NSTAGE * STAGE_BYTES;
+  static constexpr uint32_t OFF_XW = OFF_M + 2 * kPanel;
+  static constexpr uint32_t OFF_HB = OFF_XW + kPanel;
+  static constexpr uint32_t OFF_SMALL = OFF_HB + NPAD * 128;
+  static constexpr uint32_t OFF_CS = OFF_SMALL;          // float[2][128]
+  static constexpr uint32_t OFF_DL = OFF_CS + 1024;      // float[2][128]
+  static constexpr uint32_t OFF_WS = OFF_DL + 1024;      // float[8] scan scratch + flags
+  static constexpr uint32_t OFF_BAR = OFF_WS + 64;       // 16 mbarriers
+  static constexpr uint32_t OFF_TMEM = OFF_BAR + 128;    // u32 TMEM base
+  static constexpr uint32_t SMEM = OFF_TMEM + 64;
+  // TMEM columns
+  static constexpr uint32_t COL_Z = 0, COL_YOFF = 128, COL_YDIAG = 256, COL_H = 384;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t TX_BYTES = X_BYTES + 2 * BC_BYTES;
+};
+static_assert(Cfg<1>::SMEM <= 232448, "smem budget");
+static_assert(Cfg<2>::SMEM <= 232448, "smem budget");
+static_assert(Cfg<2>::COL_H + 64 * 2 <= 512, "tmem budget");
+
+enum Bar {
+  FULL0 = 0, FULL1, EMPTY0, EMPTY1, CB_DONE, Z_FREE, PREP, STATE_DONE, M_READY,
+  YDONE0, YDONE1, YFREE0, YFREE1, TEARDOWN, NBAR
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t a) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(a), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// 32 consecutive TMEM columns of this warp's 32 lanes -> 32 registers per thread
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tc_st32(uint32_t taddr, const float* v) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
+                                       int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
+                                       int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z,
+                                             uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z),
+               "r"(w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+
+// byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128B-swizzled panel
+__device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c) {
+  return r * 128u + ((c ^ (r & 7u)) << 4);
+}
+
+// tcgen05 shared-memory matrix descriptor, 128-byte swizzle (sm100 layout type 2)
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// instruction descriptor: bf16 x bf16 -> f32, M x N, operand majorness
+__host__ __device__ constexpr uint32_t idesc(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+struct KParams {
+  Geom g;
+  const void* dt;
+  const float* A;
+  const float* D;
+  const float* dt_bias;
+  const float* init;
+  const int32_t* cu;
+  __nv_bfloat16* y;
+  float* final_states;
+  int* status;
+  int units;
+  int pslices;
+};
+
+struct Unit {
+  int d, h, ps;
+  int64_t start;
+  int len, ntiles;
+};
+
+__device__ __forceinline__ Unit unit_of(const KParams& k, int u) {
+  Unit U;
+  U.ps = u % k.pslices;
+  const int t = u / k.pslices;
+  U.h = t % k.g.H;
+  U.d = t / k.g.H;
+  if (k.g.varlen) {
+    U.start = k.cu[U.d];
+    U.len = (int)((int64_t)k.cu[U.d + 1] - U.start);
+  } else {
+    U.start = (int64_t)U.d * k.g.seqlen;
+    U.len = (int)k.g.seqlen;
+  }
+  U.ntiles = (U.len + kTile - 1) / kTile;
+  return U;
+}
+
+// Bounded wait: false (and the abort flag raised) if the phase did not complete
+// within ~2 s or another role already gave up.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int* status) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  uint32_t n = 0;
+  while (!mbar_try(bar, parity)) {
+    if ((++n & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > 2000000000ull) {
+        *abort_flag = 1;
+        set_status(status, SSD_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    ssd_tc_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+                 const __grid_constant__ CUtensorMap tm_c, const KParams kp) {
+  using C = Cfg<NT>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = su32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* cs_s = reinterpret_cast<float*>(smem + C::OFF_CS);  // [2][128] cs * log2(e)
+  float* dl_s = reinterpret_cast<float*>(smem + C::OFF_DL);  // [2][128] delta
+  float* wsum = reinterpret_cast<float*>(smem + C::OFF_WS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_WS + 32);
+  int* bad_flag = reinterpret_cast<int*>(smem + C::OFF_WS + 36);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
+  auto bar = [&](int i) { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
+  const Geom& g = kp.g;
+
+  // ---- set-up: alignment check, cu_seqlens check, barriers, TMEM ----------------
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    *bad_flag = (sbase & 1023u) != 0 ? 2 : 0;
+  }
+  __syncthreads();
+  if (g.varlen) {
+    int bad = 0;
+    for (int d = threadIdx.x; d <= g.ndocs; d += kThreads) {
+      const int64_t v = kp.cu[d];
+      if (d == 0 && v != 0) bad = 1;
+      if (d == g.ndocs && v != g.tokens) bad = 1;
+      if (d > 0 && v < (int64_t)kp.cu[d - 1]) bad = 1;
+    }
+    if (bad) atomicOr(bad_flag, 1);
+  }
+  __syncthreads();
+  if (*bad_flag) {
+    if (threadIdx.x == 0)
+      set_status(kp.status, (*bad_flag & 1) ? SSD_ERR_BAD_SEQLENS : SSD_ERR_INVALID_ARG);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar(FULL0), 1);
+    mbar_init(bar(FULL1), 1);
+    mbar_init(bar(EMPTY0), 1);
+    mbar_init(bar(EMPTY1), 1);
+    mbar_init(bar(CB_DONE), 1);
+    mbar_init(bar(Z_FREE), 128);
+    mbar_init(bar(PREP), 128);
+    mbar_init(bar(STATE_DONE), 1);
+    mbar_init(bar(M_READY), 128);
+    mbar_init(bar(YDONE0), 1);
+    mbar_init(bar(YDONE1), 1);
+    mbar_init(bar(YFREE0), 128);
+    mbar_init(bar(YFREE1), 128);
+    mbar_init(bar(TEARDOWN), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     su32(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ================================ TMA producer ================================
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool issued_any = false;
+      for (int u = blockIdx.x; u < kp.units && !*abort_flag; u += gridDim.x) {
+        const Unit U = unit_of(kp, u);
+        const int g_idx = U.h / (g.H / g.G);
+        const int xcol = U.h * g.P + U.ps * kPT;
+        for (int jt = 0; jt < U.ntiles; ++jt, ++it) {
+          const uint32_t s = it % C::NSTAGE, k = it / C::NSTAGE;
+          if (k > 0 && !wait_bar(bar(EMPTY0 + s), (k - 1) & 1, abort_flag, kp.status)) break;
+          const uint32_t st = sbase + s * C::STAGE_BYTES;
+          const uint32_t fb = bar(FULL0 + s);
+          mbar_expect_tx(fb, C::TX_BYTES);
+          const int t0 = (int)(U.start + (int64_t)jt * kTile);
+          issued_any = true;
+          tma_2d(st, &tm_x, fb, xcol, t0);
+#pragma unroll
+          for (int q = 0; q < C::NPANEL; ++q) {
+            tma_3d(st + C::X_BYTES + q * kPanel, &tm_b, fb, q * 64, g_idx, t0);
+            tma_3d(st + C::X_BYTES + C::BC_BYTES + q * kPanel, &tm_c, fb, q * 64, g_idx, t0);
+          }
+        }
+      }
+      // drain: the last fill of every stage must have landed before the CTA can exit
+      // (already true on the normal path; bounded to ~0.1 s on an aborted one)
+      if (issued_any) {
+        for (uint32_t s = 0; s < C::NSTAGE; ++s) {
+          if (it <= s) continue;
+          const uint32_t last = (it - 1 - s) / C::NSTAGE * C::NSTAGE + s;  // last tile using s
+          const uint32_t k = last / C::NSTAGE;
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try(bar(FULL0 + s), k & 1) && globaltimer() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================================ MMA issuer =================================
+    if (lane == 0) {
+      constexpr uint32_t ID_CB = idesc(128, 128, 0, 0);   // Z = C B^T
+      constexpr uint32_t ID_YOFF = idesc(128, kPT, 0, 1); // Yoff = C Hb   (Hb MN-major)
+      constexpr uint32_t ID_ST = idesc(128, kPT, 1, 1);   // H += B^T XW   (both MN-major)
+      constexpr uint32_t ID_YD = idesc(128, kPT, 0, 1);   // Ydiag = M X   (X MN-major)
+      const uint32_t m_base = sbase + C::OFF_M, xw_base = sbase + C::OFF_XW,
+                     hb_base = sbase + C::OFF_HB;
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < kp.units && ok; u += gridDim.x) {
+        const Unit U = unit_of(kp, u);
+        for (int jt = 0; jt < U.ntiles; ++jt, ++it) {
+          const uint32_t s = it % C::NSTAGE, k = it / C::NSTAGE;
+          const uint32_t st = sbase + s * C::STAGE_BYTES;
+          const uint32_t x_base = st, b_base = st + C::X_BYTES, c_base = st + C::X_BYTES + C::BC_BYTES;
+          const uint32_t yb = it & 1;
+          ok = wait_bar(bar(FULL0 + s), k & 1, abort_flag, kp.status);
+          if (ok && it > 0) ok = wait_bar(bar(Z_FREE), (it - 1) & 1, abort_flag, kp.status);
+          if (!ok) break;
+          tc_fence_after();
+          // Z = C_j B_j^T : K = state dim, both operands K-major
+#pragma unroll
+          for (int kk = 0; kk < C::NPAD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+            tc_mma(tmem + C::COL_Z, sdesc(c_base + off, 16, 1024), sdesc(b_base + off, 16, 1024),
+                   ID_CB, kk > 0);
+          }
+          tc_commit(bar(CB_DONE));
+          ok = wait_bar(bar(PREP), it & 1, abort_flag, kp.status);
+          if (ok && it >= 2) ok = wait_bar(bar(YFREE0 + yb), ((it - 2) >> 1) & 1, abort_flag, kp.status);
+          if (!ok) break;
+          tc_fence_after();
+          // Yoff = C_j Hb : K = state dim; Hb rows are n (K), 128 B of p (MN)
+#pragma unroll
+          for (int kk = 0; kk < C::NPAD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+            tc_mma(tmem + C::COL_YOFF + yb * kPT, sdesc(c_base + off, 16, 1024),
+                   sdesc(hb_base + kk * 2048, C::NPAD * 128, 1024), ID_YOFF, kk > 0);
+          }
+          // H += B_j^T XW : K = tokens; A = B tile read MN-major (n), B = XW MN-major (p)
+#pragma unroll
+          for (int mt = 0; mt < NT; ++mt) {
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              tc_mma(tmem + C::COL_H + mt * kPT,
+                     sdesc(b_base + 2 * mt * kPanel + kk * 2048, kPanel, 1024),
+                     sdesc(xw_base + kk * 2048, kPanel, 1024), ID_ST, 1);
+            }
+          }
+          tc_commit(bar(STATE_DONE));
+          ok = wait_bar(bar(M_READY), it & 1, abort_flag, kp.status);
+          if (!ok) break;
+          tc_fence_after();
+          // Ydiag = M X_j : K = tokens; M K-major (2 panels), X MN-major
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+            tc_mma(tmem + C::COL_YDIAG + yb * kPT, sdesc(m_base + off, 16, 1024),
+                   sdesc(x_base + kk * 2048, kPanel, 1024), ID_YD, kk > 0);
+          }
+          tc_commit(bar(YDONE0 + yb));
+          tc_commit(bar(EMPTY0 + s));
+        }
+      }
+      // every MMA this thread issued has completed once TEARDOWN fires
+      tc_commit(bar(TEARDOWN));
+      wait_bar(bar(TEARDOWN), 0, abort_flag, kp.status);
+    }
+  } else {
+    // ================================ epilogue (warps 2..5) =======================
+    const int q = warp & 3;            // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;       // tile row (token) == TMEM lane
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const float LOG2E = 1.4426950408889634f;
+    const uint32_t m_base = sbase + C::OFF_M, xw_base = sbase + C::OFF_XW,
+                   hb_base = sbase + C::OFF_HB;
+    uint32_t it = 0;
+    bool ok = true;
+    // previous tile (its outputs are written one tile late) and pending final state
+    bool prev = false;
+    int64_t prev_t0 = 0;
+    int prev_len = 0, prev_h = 0, prev_ps = 0;
+    bool pend = false;
+    int pend_d = 0, pend_h = 0, pend_ps = 0;
+
+    auto store_final = [&](int d, int h, int ps, int n, const float* v) {
+      if (!kp.final_states || n >= g.N) return;
+      float* dst = kp.final_states + (((int64_t)d * g.H + h) * g.N + n) * g.P + ps * kPT;
+#pragma unroll
+      for (int c = 0; c < kPT; c += 4)
+        *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+    };
+    // output of tile (it-1): y = exp(cs) Yoff + Ydiag
+    auto emit_prev = [&](uint32_t pit) -> bool {
+      const uint32_t yb = pit & 1;
+      if (!wait_bar(bar(YDONE0 + yb), (pit >> 1) & 1, abort_flag, kp.status)) return false;
+      tc_fence_after();
+      const float sc = ex2(cs_s[(pit & 1) * 128 + r]);
+      const bool valid = r < prev_len;
+      __nv_bfloat16* dst = kp.y + ((prev_t0 + r) * g.H + prev_h) * (int64_t)g.P + prev_ps * kPT;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float yo[32], yd[32];
+        tc_ld32(tmem + lane_off + C::COL_YOFF + yb * kPT + half * 32, yo);
+        tc_ld32(tmem + lane_off + C::COL_YDIAG + yb * kPT + half * 32, yd);
+        tc_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint4 v;
+            v.x = pack_bf16(fmaf(sc, yo[c + 0], yd[c + 0]), fmaf(sc, yo[c + 1], yd[c + 1]));
+            v.y = pack_bf16(fmaf(sc, yo[c + 2], yd[c + 2]), fmaf(sc, yo[c + 3], yd[c + 3]));
+            v.z = pack_bf16(fmaf(sc, yo[c + 4], yd[c + 4]), fmaf(sc, yo[c + 5], yd[c + 5]));
+            v.w = pack_bf16(fmaf(sc, yo[c + 6], yd[c + 6]), fmaf(sc, yo[c + 7], yd[c + 7]));
+            *reinterpret_cast<uint4*>(dst + half * 32 + c) = v;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(YFREE0 + yb));
+      return true;
+    };
+
+    for (int u = blockIdx.x; u < kp.units && ok; u += gridDim.x) {
+      const Unit U = unit_of(kp, u);
+      if (U.ntiles == 0) {  // empty document: the final state is the initial state
+        for (int mt = 0; mt < NT; ++mt) {
+          const int n = r + 128 * mt;
+          if (n >= g.N || !kp.final_states) continue;
+          float v[kPT];
+          const float* src = kp.init ? kp.init + (((int64_t)U.d * g.H + U.h) * g.N + n) * g.P + U.ps * kPT
+                                     : nullptr;
+#pragma unroll
+          for (int c = 0; c < kPT; ++c) v[c] = src ? src[c] : 0.f;
+          store_final(U.d, U.h, U.ps, n, v);
+        }
+        continue;
+      }
+      const float Ah = kp.A[U.h];
+      const float bias = kp.dt_bias ? kp.dt_bias[U.h] : 0.f;
+      const float Dh = kp.D ? kp.D[U.h] : 0.f;
+      for (int jt = 0; jt < U.ntiles && ok; ++jt, ++it) {
+        const int64_t t0 = U.start + (int64_t)jt * kTile;
+        const int len = min(kTile, U.len - jt * kTile);
+        const uint32_t s = it % C::NSTAGE, k = it / C::NSTAGE;
+        const uint32_t cb = (it & 1) * 128;
+        // ---- E1: delta and in-tile cumulative log decay (scaled by log2 e) ----
+        float dl = 0.f, la = 0.f;
+        if (r < len) {
+          const float z = load_f(kp.dt, (t0 + r) * g.H + U.h, 1) + bias;
+          dl = softplus_f(z);
+          la = dl * Ah * LOG2E;
+        }
+        float v = la;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float t = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += t;
+        }
+        epi_sync();  // previous readers of wsum / cs slot are done
+        if (lane == 31) wsum[q] = v;
+        epi_sync();
+        for (int w = 0; w < q; ++w) v += wsum[w];
+        cs_s[cb + r] = v;
+        dl_s[cb + r] = dl;
+        epi_sync();
+        const float cs_last = cs_s[cb + 127];
+        const float cs_r = v;
+
+        // ---- E3: state entering the tile -> bf16 copy (Hb), decayed copy in TMEM ----
+        if (it > 0) ok = wait_bar(bar(STATE_DONE), (it - 1) & 1, abort_flag, kp.status);
+        if (!ok) break;
+        tc_fence_after();
+        const float decay = ex2(cs_last);
+#pragma unroll
+        for (int mt = 0; mt < NT; ++mt) {
+          const int n = r + 128 * mt;
+          const uint32_t th = tmem + lane_off + C::COL_H + mt * kPT;
+          float hv[kPT];
+          if (jt == 0) {
+            if (pend) {
+              tc_ld32(th, hv);
+              tc_ld32(th + 32, hv + 32);
+              tc_wait_ld();
+              store_final(pend_d, pend_h, pend_ps, n, hv);
+            }
+            const float* src = (kp.init && n < g.N)
+                                   ? kp.init + (((int64_t)U.d * g.H + U.h) * g.N + n) * g.P + U.ps * kPT
+                                   : nullptr;
+#pragma unroll
+            for (int c = 0; c < kPT; c += 4) {
+              float4 f = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0, 0, 0, 0);
+              hv[c] = f.x;
+              hv[c + 1] = f.y;
+              hv[c + 2] = f.z;
+              hv[c + 3] = f.w;
+            }
+          } else {
+            tc_ld32(th, hv);
+            tc_ld32(th + 32, hv + 32);
+            tc_wait_ld();
+          }
+          // Hb row n (MN-major operand of Yoff: rows = n, 128 bytes of p per row)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            st_shared_v4(hb_base + swz((uint32_t)n, (uint32_t)c),
+                         pack_bf16(hv[8 * c + 0], hv[8 * c + 1]), pack_bf16(hv[8 * c + 2], hv[8 * c + 3]),
+                         pack_bf16(hv[8 * c + 4], hv[8 * c + 5]), pack_bf16(hv[8 * c + 6], hv[8 * c + 7]));
+          }
+#pragma unroll
+          for (int c = 0; c < kPT; ++c) hv[c] *= decay;
+          tc_st32(th, hv);
+          tc_st32(th + 32, hv + 32);
+        }
+        pend = false;
+        tc_wait_st();
+
+        // ---- E4: XW = w o x_j,  w_s = exp(cs_last - cs_s) delta_s ----
+        ok = wait_bar(bar(FULL0 + s), k & 1, abort_flag, kp.status);
+        if (!ok) break;
+        {
+          const float wr = ex2(cs_last - cs_r) * dl;
+          const uint32_t xrow = sbase + s * C::STAGE_BYTES;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 xv = ld_shared_v4(xrow + swz((uint32_t)r, (uint32_t)c));
+            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+            float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
+            float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
+            st_shared_v4(xw_base + swz((uint32_t)r, (uint32_t)c), pack_bf16(wr * f0.x, wr * f0.y),
+                         pack_bf16(wr * f1.x, wr * f1.y), pack_bf16(wr * f2.x, wr * f2.y),
+                         pack_bf16(wr * f3.x, wr * f3.y));
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(PREP));
+
+        // ---- E2: decay mask of the diagonal block -> M (bf16, K-major) ----
+        ok = wait_bar(bar(CB_DONE), it & 1, abort_flag, kp.status);
+        if (ok && it > 0) ok = wait_bar(bar(YDONE0 + ((it - 1) & 1)), ((it - 1) >> 1) & 1, abort_flag,
+                                        kp.status);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t panel = m_base + (uint32_t)(cc >> 1) * kPanel;
+          if (cc > q) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              st_shared_v4(panel + swz((uint32_t)r, (uint32_t)((cc & 1) * 4 + i)), 0u, 0u, 0u, 0u);
+            continue;
+          }
+          float zv[32];
+          tc_ld32(tmem + lane_off + C::COL_Z + cc * 32, zv);
+          tc_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int sidx = cc * 32 + j;
+            float m = zv[j] * ex2(cs_r - cs_s[cb + sidx]) * dl_s[cb + sidx];
+            if (sidx == r) m += Dh;
+            zv[j] = sidx <= r ? m : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            st_shared_v4(panel + swz((uint32_t)r, (uint32_t)((cc & 1) * 4 + i)),
+                         pack_bf16(zv[8 * i + 0], zv[8 * i + 1]), pack_bf16(zv[8 * i + 2], zv[8 * i + 3]),
+                         pack_bf16(zv[8 * i + 4], zv[8 * i + 5]), pack_bf16(zv[8 * i + 6], zv[8 * i + 7]));
+        }
+        tc_fence_before();
+        mbar_arrive(bar(Z_FREE));
+        fence_async_smem();
+        mbar_arrive(bar(M_READY));
+
+        // ---- E5 of the previous tile ----
+        if (prev) {
+          if (!emit_prev(it - 1)) {
+            ok = false;
+            break;
+          }
+        }
+        prev = true;
+        prev_t0 = t0;
+        prev_len = len;
+        prev_h = U.h;
+        prev_ps = U.ps;
+        if (jt == U.ntiles - 1) {
+          pend = true;
+          pend_d = U.d;
+          pend_h = U.h;
+          pend_ps = U.ps;
+        }
+      }
+    }
+    if (ok && prev) ok = emit_prev(it - 1);
+    if (ok && pend) {
+      ok = wait_bar(bar(STATE_DONE), (it - 1) & 1, abort_flag, kp.status);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int mt = 0; mt < NT; ++mt) {
+          float hv[kPT];
+          const uint32_t th = tmem + lane_off + C::COL_H + mt * kPT;
+          tc_ld32(th, hv);
+          tc_ld32(th + 32, hv + 32);
+          tc_wait_ld();
+          store_final(pend_d, pend_h, pend_ps, r + 128 * mt, hv);
+        }
+      }
+    }
+  }
+
+  // ---- teardown ----
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tc_supported(const Geom& g, const Args*) {
+  if (!g.in_bf16 || !g.out_bf16) return false;
+  if (g.tokens <= 0 || g.tokens > 0x7fffffffLL || g.ndocs < 1) return false;
+  if (g.P % kPT != 0 || g.P > 256) return false;
+  if (g.N < 16 || g.N > 256 || g.N % 16 != 0) return false;
+  if (g.Q % kTile != 0) return false;
+  if ((int64_t)g.ndocs * g.H * (g.P / kPT) > 0x7fffffff) return false;
+  return true;
+}
+
+int tc_units(const Geom& g) { return g.ndocs * g.H * (g.P / kPT); }
+int tc_kernels(const Geom&) { return 1; }
+size_t tc_workspace_bytes(const Geom&) { return 256; }
+
+cudaError_t tc_forward(const Geom& g, const Args& a, void*, int* status, cudaStream_t stream,
+                       int num_sms) {
+  CUtensorMap tx, tb, tc;
+  const cuuint64_t T = (cuuint64_t)g.tokens;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)g.H * g.P, T};
+    cuuint64_t str[1] = {(cuuint64_t)g.H * g.P * 2};
+    cuuint32_t box[2] = {64, kTile};
+    if (!encode(&tx, a.x, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)g.N, (cuuint64_t)g.G, T};
+    cuuint64_t str[2] = {(cuuint64_t)g.N * 2, (cuuint64_t)g.G * g.N * 2};
+    cuuint32_t box[3] = {64, 1, kTile};
+    if (!encode(&tb, a.B, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!encode(&tc, a.C, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  KParams kp;
+  kp.g = g;
+  kp.dt = a.dt;
+  kp.A = a.A;
+  kp.D = a.D;
+  kp.dt_bias = a.dt_bias;
+  kp.init = a.init;
+  kp.cu = a.cu;
+  kp.y = reinterpret_cast<__nv_bfloat16*>(a.y);
+  kp.final_states = a.final_states;
+  kp.status = status;
+  kp.pslices = g.P / kPT;
+  kp.units = tc_units(g);
+  const int grid = kp.units < num_sms ? kp.units : num_sms;
+  if (g.N <= 128) {
+    cudaError_t e = cudaFuncSetAttribute(ssd_tc_fused<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg<1>::SMEM);
+    if (e != cudaSuccess) return e;
+    ssd_tc_fused<1><<<grid, kThreads, Cfg<1>::SMEM, stream>>>(tx, tb, tc, kp);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(ssd_tc_fused<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg<2>::SMEM);
+    if (e != cudaSuccess) return e;
+    ssd_tc_fused<2><<<grid, kThreads, Cfg<2>::SMEM, stream>>>(tx, tb, tc, kp);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ssd
