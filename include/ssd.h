@@ -65,7 +65,8 @@ enum {
   SSD_ERR_CUDA = -3,        /* a CUDA runtime call or kernel launch failed */
   SSD_ERR_TIMEOUT = -4,     /* a device-side bounded wait gave up (status word) */
   SSD_ERR_OOM = -5,         /* device allocation failed */
-  SSD_ERR_BAD_SEQLENS = -6  /* cu_seqlens not 0 = c[0] <= ... <= c[n] = tokens (status word) */
+  SSD_ERR_BAD_SEQLENS = -6, /* cu_seqlens not 0 = c[0] <= ... <= c[n] = tokens (status word) */
+  SSD_ERR_SCRATCH_TOO_SMALL = -7 /* ssd_forward_noalloc: problem needs more than its fixed scratch */
 };
 
 /* kernel paths (ssd_plan_t.path, SSD_OPT_FORCE_PATH) */
@@ -195,6 +196,45 @@ SSD_API int ssd_get_status(ssd_handle_t h, ssd_stream_t stream);
 
 /* ssd_destroy: synchronises the device and frees everything the handle owns. NULL is a no-op. */
 SSD_API int ssd_destroy(ssd_handle_t h);
+
+/*
+ * ssd_forward_noalloc: ssd_forward for callers that may not allocate device memory.
+ * The paper has no counterpart to this entry point; it exists for deployment.
+ *
+ * Some callers cannot call cudaMalloc on the path that runs the layer: an
+ * application that budgets all device memory up front through its own allocator,
+ * or code that cannot afford the device-wide synchronisation an allocation may
+ * cause.  This entry point takes no handle and allocates nothing.  The caller
+ * passes every input and output exactly as for ssd_forward (same layouts,
+ * alignment and stream semantics; `desc` describes the problem).  The computation
+ * is the chunk-parallel CUDA-core path (the kernels ssd_forward runs with
+ * SSD_PATH_SIMT) and gives its results.
+ *
+ * Its scratch memory is one fixed device array of SSD_NOALLOC_SCRATCH_BYTES
+ * (32 MiB) inside the library, reserved on every device where the library's
+ * kernels are loaded and held until the process exits.  A problem whose scratch
+ * would exceed it (about chunks x H x N x P x 4 bytes plus 8 bytes per token and
+ * head) is refused with SSD_ERR_SCRATCH_TOO_SMALL before any work is enqueued.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  All calls on a device share the one array and the previous
+ * call's contents stay in it (nothing needs to start at zero), so calls whose GPU
+ * work overlaps -- on different streams without ordering -- race and must be
+ * serialised by the caller.
+ *
+ *   status   optional device int (NULL: none).  Set to 0 on `stream` at the start
+ *            of the call; a device-side error (an invalid cu_seqlens array,
+ *            SSD_ERR_BAD_SEQLENS) is written there, and then no output is written.
+ * Returns SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED,
+ * SSD_ERR_SCRATCH_TOO_SMALL or SSD_ERR_CUDA (launch failure).
+ */
+#define SSD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+SSD_API int ssd_forward_noalloc(const ssd_desc_t* desc, const void* x, const void* dt,
+                                const float* A, const void* B, const void* C, const float* D,
+                                const float* dt_bias, int chunk_size, const float* initial_states,
+                                const int32_t* cu_seqlens, int num_docs, void* y,
+                                float* final_states, int* status, ssd_stream_t stream);
 
 /* Static string naming a return code. */
 SSD_API const char* ssd_error_string(int code);

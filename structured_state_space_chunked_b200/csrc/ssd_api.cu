@@ -323,6 +323,8 @@ const char* ssd_error_string(int code) {
     case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: a device-side wait gave up";
     case SSD_ERR_OOM: return "SSD_ERR_OOM: device allocation failed";
     case SSD_ERR_BAD_SEQLENS: return "SSD_ERR_BAD_SEQLENS: cu_seqlens is not a valid partition";
+    case SSD_ERR_SCRATCH_TOO_SMALL:
+      return "SSD_ERR_SCRATCH_TOO_SMALL: the problem needs more scratch than the fixed array";
     default: return "SSD_ERR_UNKNOWN";
   }
 }

@@ -23,12 +23,15 @@ SSD_OPT_FORCE_PATH = 1
 ERRORS = {
     0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3: "SSD_ERR_CUDA",
     -4: "SSD_ERR_TIMEOUT", -5: "SSD_ERR_OOM", -6: "SSD_ERR_BAD_SEQLENS",
+    -7: "SSD_ERR_SCRATCH_TOO_SMALL",
 }
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 # every symbol include/ssd.h declares
 ABI_SYMBOLS = (
     "ssd_validate_desc", "ssd_plan", "ssd_create", "ssd_set_option", "ssd_forward",
     "ssd_forward_host", "ssd_get_status", "ssd_destroy", "ssd_error_string", "ssd_version",
+    "ssd_forward_noalloc",
 )
 
 
@@ -76,6 +79,9 @@ def lib():
         L.ssd_forward.argtypes = fwd
         L.ssd_forward_host.argtypes = fwd
         L.ssd_get_status.argtypes = [vp, vp]
+        L.ssd_forward_noalloc.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp, vp, i32,
+                                          vp, vp, i32, vp, vp, vp, vp]
+        L.ssd_forward_noalloc.restype = ctypes.c_int
         L.ssd_destroy.argtypes = [vp]
         L.ssd_error_string.argtypes = [i32]
         L.ssd_error_string.restype = ctypes.c_char_p
