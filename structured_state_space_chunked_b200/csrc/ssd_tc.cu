@@ -27,10 +27,13 @@
 // a strictly lower block is rank one, §3.2.2), which equals the quadratic form
 // up to rounding.
 //
-// Roles: warp 0 issues TMA loads (double-buffered x/B/C tiles), warp 1 owns TMEM
-// and one thread issues every tcgen05.mma, warps 2..5 are the epilogue
-// (cumsum, decay mask, state rescale, outputs).  Every mbarrier wait is bounded:
-// on expiry the CTA records SSD_ERR_TIMEOUT in the status word and unwinds.
+// Roles: warp 0 issues TMA loads (x/B/C tiles, double-buffered when they fit),
+// warp 1 owns TMEM and one thread issues every tcgen05.mma, warps 2..5
+// (epilogue A) compute the cumulative decay, hand the state over and build the
+// decay-masked operand M in TMEM (over C B^T, as bf16), warps 6..9 (epilogue B)
+// build the weighted input w o x and write the outputs.  The two epilogue groups
+// work on consecutive tiles at once.  Every mbarrier wait is bounded: on expiry
+// the CTA records SSD_ERR_TIMEOUT in the status word and unwinds.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -40,31 +43,35 @@
 namespace ssd {
 namespace {
 
-constexpr int kTile = 128;     // tokens per tile
-constexpr int kPT = 64;        // head-dim columns per unit
-constexpr int kThreads = 192;  // 6 warps
+constexpr int kTile = 128;          // tokens per tile
+constexpr int kPT = 64;             // head-dim columns per unit
+constexpr int kThreads = 320;       // 10 warps: TMA, MMA, epilogue A (4), epilogue B (4)
 constexpr uint32_t kPanel = 16384;  // one 128-row x 128-byte SW128 panel
 
 template <int NT>
 struct Cfg {
-  static constexpr int NPAD = 128 * NT;        // state dim padded to the lane tiles
+  static constexpr int NPAD = 128 * NT;        // state dim padded to whole lane tiles
   static constexpr int NPANEL = 2 * NT;        // 64-column panels of a B/C tile
   static constexpr int NSTAGE = NT == 1 ? 2 : 1;
+  static constexpr int HB_BUFS = NT == 1 ? 2 : 1;
   static constexpr uint32_t X_BYTES = kPanel;
   static constexpr uint32_t BC_BYTES = NPANEL * kPanel;
   static constexpr uint32_t STAGE_BYTES = X_BYTES + 2 * BC_BYTES;
-  static constexpr uint32_t OFF_M = NSTAGE * STAGE_BYTES;
-  static constexpr uint32_t OFF_XW = OFF_M + 2 * kPanel;
+  static constexpr uint32_t HB_BYTES = NPAD * 128;
+  static constexpr uint32_t OFF_XW = NSTAGE * STAGE_BYTES;
   static constexpr uint32_t OFF_HB = OFF_XW + kPanel;
-  static constexpr uint32_t OFF_SMALL = OFF_HB + NPAD * 128;
-  static constexpr uint32_t OFF_CS = OFF_SMALL;          // float[2][128]
-  static constexpr uint32_t OFF_DL = OFF_CS + 1024;      // float[2][128]
-  static constexpr uint32_t OFF_WS = OFF_DL + 1024;      // float[8] scan scratch + flags
-  static constexpr uint32_t OFF_BAR = OFF_WS + 64;       // 16 mbarriers
-  static constexpr uint32_t OFF_TMEM = OFF_BAR + 128;    // u32 TMEM base
+  static constexpr uint32_t OFF_SMALL = OFF_HB + HB_BUFS * HB_BYTES;
+  static constexpr uint32_t OFF_CS = OFF_SMALL;       // float[2][128]  cs * log2(e)
+  static constexpr uint32_t OFF_DL = OFF_CS + 1024;   // float[2][128]  delta
+  static constexpr uint32_t OFF_V = OFF_DL + 1024;    // float[2][128]  exp(cs_blockend - cs) delta
+  static constexpr uint32_t OFF_W = OFF_V + 1024;     // float[2][128]  exp(cs_last - cs) delta
+  static constexpr uint32_t OFF_WS = OFF_W + 1024;    // scan scratch [2][4] and flags
+  static constexpr uint32_t OFF_BAR = OFF_WS + 64;    // mbarriers
+  static constexpr uint32_t OFF_TMEM = OFF_BAR + 256;
   static constexpr uint32_t SMEM = OFF_TMEM + 64;
-  // TMEM columns
-  static constexpr uint32_t COL_Z = 0, COL_YOFF = 128, COL_YDIAG = 256, COL_H = 384;
+  // TMEM columns: two C B^T tiles (each turned in place into the bf16 mask
+  // operand M), the two output accumulators and the state (NT lane tiles)
+  static constexpr uint32_t COL_Z = 0, COL_YOFF = 256, COL_YDIAG = 320, COL_H = 384;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TX_BYTES = X_BYTES + 2 * BC_BYTES;
 };
@@ -73,8 +80,9 @@ static_assert(Cfg<2>::SMEM <= 232448, "smem budget");
 static_assert(Cfg<2>::COL_H + 64 * 2 <= 512, "tmem budget");
 
 enum Bar {
-  FULL0 = 0, FULL1, EMPTY0, EMPTY1, CB_DONE, Z_FREE, PREP, STATE_DONE, M_READY,
-  YDONE0, YDONE1, YFREE0, YFREE1, TEARDOWN, NBAR
+  FULL0 = 0, FULL1, EMPTY0, EMPTY1, CB_DONE0, CB_DONE1, STATE_DONE, HB_READY, XW_READY,
+  M_READY_A0, M_READY_A1, M_READY_B0, M_READY_B1, YDONE0, YDONE1, Y_FREE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1,
+  TEARDOWN, NBAR
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -123,12 +131,22 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                    bar)
                : "memory");
 }
+// D(tmem) (+)= A(smem desc) * B(smem desc)
 __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
                                        uint32_t accum) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+// D(tmem) (+)= A(tmem) * B(smem desc)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                          uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum)
       : "memory");
 }
 __device__ __forceinline__ void tc_wait_ld() {
@@ -162,6 +180,15 @@ __device__ __forceinline__ void tc_st32(uint32_t taddr, const float* v) {
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
                                        int c1) {
   asm volatile(
@@ -178,8 +205,12 @@ __device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* m, uint3
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
-__device__ __forceinline__ void epi_sync() {
+// named barriers of epilogue group A (warps 2..5) and group B (warps 6..9)
+__device__ __forceinline__ void sync_a() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+__device__ __forceinline__ void sync_b() {
+  asm volatile("bar.sync 2, 128;" ::: "memory");
 }
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -214,7 +245,7 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
   return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-// instruction descriptor: bf16 x bf16 -> f32, M x N, operand majorness
+// instruction descriptor: bf16 x bf16 -> f32, M x N, operand majorness (1 = MN-major)
 __host__ __device__ constexpr uint32_t idesc(int M, int N, int a_mn, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -258,6 +289,37 @@ __device__ __forceinline__ Unit unit_of(const KParams& k, int u) {
   return U;
 }
 
+// The stream of tiles a CTA processes: units blockIdx.x, +gridDim.x, ...; units
+// without tokens contribute no tile.  Every role walks the same stream.
+struct Cursor {
+  int u, jt;
+  bool valid;
+  Unit U;
+};
+__device__ __forceinline__ void cursor_next(const KParams& kp, Cursor& c) {
+  if (c.valid && c.jt + 1 < c.U.ntiles) {
+    ++c.jt;
+    return;
+  }
+  for (c.u += gridDim.x; c.u < kp.units; c.u += gridDim.x) {
+    c.U = unit_of(kp, c.u);
+    if (c.U.ntiles > 0) {
+      c.jt = 0;
+      c.valid = true;
+      return;
+    }
+  }
+  c.valid = false;
+}
+__device__ __forceinline__ Cursor cursor_first(const KParams& kp) {
+  Cursor c;
+  c.u = (int)blockIdx.x - (int)gridDim.x;
+  c.jt = 0;
+  c.valid = false;
+  cursor_next(kp, c);
+  return c;
+}
+
 // Bounded wait: false (and the abort flag raised) if the phase did not complete
 // within ~2 s or another role already gave up.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -278,6 +340,43 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   return true;
 }
 
+// Decay mask of column block cc (s in [32cc, 32cc+32)) for this thread's row r of
+// the diagonal block: reads C B^T from TMEM (Z) and writes M[r, s] as bf16 pairs
+// into the first 16 columns of the same 32-column block (in place, so any warp of
+// the lane quarter may handle any block).  Blocks left of the diagonal block use
+// exp(cs_r - cs_s) = exp(cs_r - cs_b) exp(cs_b - cs_s), b = 32cc + 31, with the
+// second factor (times delta_s) precomputed per column in v.
+__device__ __forceinline__ void mask_block(uint32_t zaddr, int cc, int q, int r, float cs_r,
+                                           const float* cs, const float* dl, const float* v,
+                                           float Dh) {
+  float zv[32];
+  tc_ld32(zaddr + 32 * cc, zv);
+  tc_wait_ld();
+  if (cc < q) {
+    const float u = ex2(cs_r - cs[32 * cc + 31]);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) zv[j] *= u * v[32 * cc + j];
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int sidx = 32 * cc + j;
+      float m = zv[j] * ex2(cs_r - cs[sidx]) * dl[sidx];
+      if (sidx == r) m += Dh;
+      zv[j] = sidx <= r ? m : 0.f;
+    }
+  }
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(zv[2 * i], zv[2 * i + 1]);
+  tc_st16(zaddr + 32 * cc, pk);
+}
+__device__ __forceinline__ void zero_block(uint32_t zaddr, int cc) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pk[i] = 0u;
+  tc_st16(zaddr + 32 * cc, pk);
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_tc_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
@@ -286,8 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = su32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* cs_s = reinterpret_cast<float*>(smem + C::OFF_CS);  // [2][128] cs * log2(e)
-  float* dl_s = reinterpret_cast<float*>(smem + C::OFF_DL);  // [2][128] delta
+  float* cs_s = reinterpret_cast<float*>(smem + C::OFF_CS);
+  float* dl_s = reinterpret_cast<float*>(smem + C::OFF_DL);
+  float* v_s = reinterpret_cast<float*>(smem + C::OFF_V);
+  float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
   float* wsum = reinterpret_cast<float*>(smem + C::OFF_WS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_WS + 32);
   int* bad_flag = reinterpret_cast<int*>(smem + C::OFF_WS + 36);
@@ -322,15 +423,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(FULL1), 1);
     mbar_init(bar(EMPTY0), 1);
     mbar_init(bar(EMPTY1), 1);
-    mbar_init(bar(CB_DONE), 1);
-    mbar_init(bar(Z_FREE), 128);
-    mbar_init(bar(PREP), 128);
+    mbar_init(bar(CB_DONE0), 1);
+    mbar_init(bar(CB_DONE1), 1);
     mbar_init(bar(STATE_DONE), 1);
-    mbar_init(bar(M_READY), 128);
+    mbar_init(bar(HB_READY), 128);
+    mbar_init(bar(XW_READY), 128);
+    mbar_init(bar(M_READY_A0), 128);
+    mbar_init(bar(M_READY_A1), 128);
+    mbar_init(bar(M_READY_B0), 128);
+    mbar_init(bar(M_READY_B1), 128);
     mbar_init(bar(YDONE0), 1);
     mbar_init(bar(YDONE1), 1);
-    mbar_init(bar(YFREE0), 128);
-    mbar_init(bar(YFREE1), 128);
+    mbar_init(bar(Y_FREE), 128);
+    mbar_init(bar(CS_READY0), 128);
+    mbar_init(bar(CS_READY1), 128);
+    mbar_init(bar(CS_FREE0), 128);
+    mbar_init(bar(CS_FREE1), 128);
     mbar_init(bar(TEARDOWN), 1);
     fence_barrier_init();
   }
@@ -350,126 +458,144 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================ TMA producer ================================
     if (lane == 0) {
       uint32_t it = 0;
-      bool issued_any = false;
-      for (int u = blockIdx.x; u < kp.units && !*abort_flag; u += gridDim.x) {
-        const Unit U = unit_of(kp, u);
-        const int g_idx = U.h / (g.H / g.G);
-        const int xcol = U.h * g.P + U.ps * kPT;
-        for (int jt = 0; jt < U.ntiles; ++jt, ++it) {
-          const uint32_t s = it % C::NSTAGE, k = it / C::NSTAGE;
-          if (k > 0 && !wait_bar(bar(EMPTY0 + s), (k - 1) & 1, abort_flag, kp.status)) break;
-          const uint32_t st = sbase + s * C::STAGE_BYTES;
-          const uint32_t fb = bar(FULL0 + s);
-          mbar_expect_tx(fb, C::TX_BYTES);
-          const int t0 = (int)(U.start + (int64_t)jt * kTile);
-          issued_any = true;
-          tma_2d(st, &tm_x, fb, xcol, t0);
+      for (Cursor c = cursor_first(kp); c.valid && !*abort_flag; cursor_next(kp, c), ++it) {
+        const uint32_t s = it % C::NSTAGE, k = it / C::NSTAGE;
+        if (k > 0 && !wait_bar(bar(EMPTY0 + s), (k - 1) & 1, abort_flag, kp.status)) break;
+        const uint32_t st = sbase + s * C::STAGE_BYTES;
+        const uint32_t fb = bar(FULL0 + s);
+        const int g_idx = c.U.h / (g.H / g.G);
+        const int t0 = (int)(c.U.start + (int64_t)c.jt * kTile);
+        mbar_expect_tx(fb, C::TX_BYTES);
+        tma_2d(st, &tm_x, fb, c.U.h * g.P + c.U.ps * kPT, t0);
 #pragma unroll
-          for (int q = 0; q < C::NPANEL; ++q) {
-            tma_3d(st + C::X_BYTES + q * kPanel, &tm_b, fb, q * 64, g_idx, t0);
-            tma_3d(st + C::X_BYTES + C::BC_BYTES + q * kPanel, &tm_c, fb, q * 64, g_idx, t0);
-          }
+        for (int q = 0; q < C::NPANEL; ++q) {
+          tma_3d(st + C::X_BYTES + q * kPanel, &tm_b, fb, q * 64, g_idx, t0);
+          tma_3d(st + C::X_BYTES + C::BC_BYTES + q * kPanel, &tm_c, fb, q * 64, g_idx, t0);
         }
       }
-      // drain: the last fill of every stage must have landed before the CTA can exit
+      // drain: the last fill of every stage must have landed before the CTA exits
       // (already true on the normal path; bounded to ~0.1 s on an aborted one)
-      if (issued_any) {
-        for (uint32_t s = 0; s < C::NSTAGE; ++s) {
-          if (it <= s) continue;
-          const uint32_t last = (it - 1 - s) / C::NSTAGE * C::NSTAGE + s;  // last tile using s
-          const uint32_t k = last / C::NSTAGE;
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try(bar(FULL0 + s), k & 1) && globaltimer() - t0 < 100000000ull) {
-          }
+      for (uint32_t s = 0; s < C::NSTAGE; ++s) {
+        if (it <= s) continue;
+        const uint32_t last = (it - 1 - s) / C::NSTAGE * C::NSTAGE + s;
+        const uint32_t k = last / C::NSTAGE;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try(bar(FULL0 + s), k & 1) && globaltimer() - t0 < 100000000ull) {
         }
       }
     }
   } else if (warp == 1) {
     // ================================ MMA issuer =================================
     if (lane == 0) {
-      constexpr uint32_t ID_CB = idesc(128, 128, 0, 0);   // Z = C B^T
-      constexpr uint32_t ID_YOFF = idesc(128, kPT, 0, 1); // Yoff = C Hb   (Hb MN-major)
-      constexpr uint32_t ID_ST = idesc(128, kPT, 1, 1);   // H += B^T XW   (both MN-major)
-      constexpr uint32_t ID_YD = idesc(128, kPT, 0, 1);   // Ydiag = M X   (X MN-major)
-      const uint32_t m_base = sbase + C::OFF_M, xw_base = sbase + C::OFF_XW,
-                     hb_base = sbase + C::OFF_HB;
+      constexpr uint32_t ID_CB = idesc(128, 128, 0, 0);    // Z = C B^T, both K-major
+      constexpr uint32_t ID_YOFF = idesc(128, kPT, 0, 1);  // Yoff = C Hb, Hb MN-major
+      constexpr uint32_t ID_ST = idesc(128, kPT, 1, 1);    // H += B^T XW, both MN-major
+      constexpr uint32_t ID_YD = idesc(128, kPT, 0, 1);    // Ydiag = M X, M in TMEM, X MN-major
+      // with two stages, C B^T of the next tile is issued before this tile's mask is
+      // ready, so the tensor cores work while the epilogue builds M
+      constexpr bool LOOKAHEAD = C::NSTAGE >= 2;
+      const uint32_t xw_base = sbase + C::OFF_XW, hb0 = sbase + C::OFF_HB;
+      auto stage_of = [&](uint32_t i) { return sbase + (i % C::NSTAGE) * C::STAGE_BYTES; };
+      // Z = C_j B_j^T for tile i (waits for its data and for its Z buffer)
+      auto issue_cb = [&](uint32_t i) -> bool {
+        const uint32_t st = stage_of(i), zb = i & 1;
+        if (!wait_bar(bar(FULL0 + i % C::NSTAGE), (i / C::NSTAGE) & 1, abort_flag, kp.status))
+          return false;
+        // Z buffer zb last held the mask operand of tile i-2
+        if (i >= 2 && !wait_bar(bar(YDONE0 + zb), ((i - 2) >> 1) & 1, abort_flag, kp.status))
+          return false;
+        tc_fence_after();
+        const uint32_t b_base = st + C::X_BYTES, c_base = st + C::X_BYTES + C::BC_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < C::NPAD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+          tc_mma(tmem + C::COL_Z + zb * 128, sdesc(c_base + off, 16, 1024),
+                 sdesc(b_base + off, 16, 1024), ID_CB, kk > 0);
+        }
+        tc_commit(bar(CB_DONE0 + zb));
+        return true;
+      };
       uint32_t it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < kp.units && ok; u += gridDim.x) {
-        const Unit U = unit_of(kp, u);
-        for (int jt = 0; jt < U.ntiles; ++jt, ++it) {
-          const uint32_t s = it % C::NSTAGE, k = it / C::NSTAGE;
-          const uint32_t st = sbase + s * C::STAGE_BYTES;
-          const uint32_t x_base = st, b_base = st + C::X_BYTES, c_base = st + C::X_BYTES + C::BC_BYTES;
-          const uint32_t yb = it & 1;
-          ok = wait_bar(bar(FULL0 + s), k & 1, abort_flag, kp.status);
-          if (ok && it > 0) ok = wait_bar(bar(Z_FREE), (it - 1) & 1, abort_flag, kp.status);
-          if (!ok) break;
-          tc_fence_after();
-          // Z = C_j B_j^T : K = state dim, both operands K-major
+      Cursor c = cursor_first(kp);
+      if (c.valid && LOOKAHEAD) ok = issue_cb(0);
+      for (; c.valid && ok; ++it) {
+        Cursor n = c;
+        cursor_next(kp, n);
+        const uint32_t s = it % C::NSTAGE, zb = it & 1;
+        const uint32_t st = stage_of(it);
+        const uint32_t x_base = st, b_base = st + C::X_BYTES, c_base = st + C::X_BYTES + C::BC_BYTES;
+        const uint32_t hb_base = hb0 + (C::HB_BUFS == 2 ? zb : 0) * C::HB_BYTES;
+        if (!LOOKAHEAD && !(ok = issue_cb(it))) break;
+        ok = wait_bar(bar(HB_READY), it & 1, abort_flag, kp.status);
+        if (ok) ok = wait_bar(bar(XW_READY), it & 1, abort_flag, kp.status);
+        if (!ok) break;
+        tc_fence_after();
+        auto issue_state = [&]() {
+          // H += B_j^T XW : K = tokens; A = the B tile read MN-major (n), B = XW MN-major (p)
 #pragma unroll
-          for (int kk = 0; kk < C::NPAD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-            tc_mma(tmem + C::COL_Z, sdesc(c_base + off, 16, 1024), sdesc(b_base + off, 16, 1024),
-                   ID_CB, kk > 0);
-          }
-          tc_commit(bar(CB_DONE));
-          ok = wait_bar(bar(PREP), it & 1, abort_flag, kp.status);
-          if (ok && it >= 2) ok = wait_bar(bar(YFREE0 + yb), ((it - 2) >> 1) & 1, abort_flag, kp.status);
-          if (!ok) break;
-          tc_fence_after();
-          // Yoff = C_j Hb : K = state dim; Hb rows are n (K), 128 B of p (MN)
+          for (int mt = 0; mt < NT; ++mt)
 #pragma unroll
-          for (int kk = 0; kk < C::NPAD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-            tc_mma(tmem + C::COL_YOFF + yb * kPT, sdesc(c_base + off, 16, 1024),
-                   sdesc(hb_base + kk * 2048, C::NPAD * 128, 1024), ID_YOFF, kk > 0);
-          }
-          // H += B_j^T XW : K = tokens; A = B tile read MN-major (n), B = XW MN-major (p)
-#pragma unroll
-          for (int mt = 0; mt < NT; ++mt) {
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk) {
+            for (int kk = 0; kk < kTile / 16; ++kk)
               tc_mma(tmem + C::COL_H + mt * kPT,
                      sdesc(b_base + 2 * mt * kPanel + kk * 2048, kPanel, 1024),
                      sdesc(xw_base + kk * 2048, kPanel, 1024), ID_ST, 1);
-            }
+        };
+        auto issue_yoff = [&]() {
+          // Yoff = C_j Hb : K = state dim; Hb rows are n (K), 128 bytes of p (MN)
+#pragma unroll
+          for (int kk = 0; kk < C::NPAD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
+            tc_mma(tmem + C::COL_YOFF, sdesc(c_base + off, 16, 1024),
+                   sdesc(hb_base + kk * 2048, C::HB_BYTES, 1024), ID_YOFF, kk > 0);
           }
+        };
+        if (C::HB_BUFS == 2) {
+          issue_state();
           tc_commit(bar(STATE_DONE));
-          ok = wait_bar(bar(M_READY), it & 1, abort_flag, kp.status);
+          if (LOOKAHEAD && n.valid && !(ok = issue_cb(it + 1))) break;
+          if (it >= 1) ok = wait_bar(bar(Y_FREE), (it - 1) & 1, abort_flag, kp.status);
           if (!ok) break;
           tc_fence_after();
-          // Ydiag = M X_j : K = tokens; M K-major (2 panels), X MN-major
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-            tc_mma(tmem + C::COL_YDIAG + yb * kPT, sdesc(m_base + off, 16, 1024),
-                   sdesc(x_base + kk * 2048, kPanel, 1024), ID_YD, kk > 0);
-          }
-          tc_commit(bar(YDONE0 + yb));
-          tc_commit(bar(EMPTY0 + s));
+          issue_yoff();
+        } else {
+          // one Hb buffer: Yoff must have read it before the next state copy lands
+          if (it >= 1) ok = wait_bar(bar(Y_FREE), (it - 1) & 1, abort_flag, kp.status);
+          if (!ok) break;
+          tc_fence_after();
+          issue_yoff();
+          issue_state();
+          tc_commit(bar(STATE_DONE));
+          if (LOOKAHEAD && n.valid && !(ok = issue_cb(it + 1))) break;
         }
+        // one barrier per tile parity and group: with C B^T issued a tile ahead, a
+        // group may finish the next tile's mask before this wait
+        ok = wait_bar(bar(M_READY_A0 + zb), (it >> 1) & 1, abort_flag, kp.status);
+        if (ok) ok = wait_bar(bar(M_READY_B0 + zb), (it >> 1) & 1, abort_flag, kp.status);
+        if (!ok) break;
+        tc_fence_after();
+        // Ydiag = M X_j : K = tokens.  M sits in TMEM as bf16 pairs: the 16 tokens of
+        // K step kk are columns 32 (kk/2) + 8 (kk%2) .. +8 of the Z buffer
+        const uint32_t z_col = tmem + C::COL_Z + zb * 128;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          tc_mma_ts(tmem + C::COL_YDIAG, z_col + 32 * (kk >> 1) + 8 * (kk & 1),
+                    sdesc(x_base + kk * 2048, kPanel, 1024), ID_YD, kk > 0);
+        tc_commit(bar(YDONE0 + zb));
+        tc_commit(bar(EMPTY0 + s));
+        c = n;
       }
       // every MMA this thread issued has completed once TEARDOWN fires
       tc_commit(bar(TEARDOWN));
       wait_bar(bar(TEARDOWN), 0, abort_flag, kp.status);
     }
-  } else {
-    // ================================ epilogue (warps 2..5) =======================
-    const int q = warp & 3;            // TMEM lane quarter of this warp
-    const int r = q * 32 + lane;       // tile row (token) == TMEM lane
+  } else if (warp < 6) {
+    // ============== epilogue A: decay, state hand-over, mask (blocks 0 and q) ==============
+    const int q = warp & 3;        // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;   // tile row (token) == TMEM lane
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float LOG2E = 1.4426950408889634f;
-    const uint32_t m_base = sbase + C::OFF_M, xw_base = sbase + C::OFF_XW,
-                   hb_base = sbase + C::OFF_HB;
-    uint32_t it = 0;
-    bool ok = true;
-    // previous tile (its outputs are written one tile late) and pending final state
-    bool prev = false;
-    int64_t prev_t0 = 0;
-    int prev_len = 0, prev_h = 0, prev_ps = 0;
-    bool pend = false;
-    int pend_d = 0, pend_h = 0, pend_ps = 0;
+    const uint32_t hb0 = sbase + C::OFF_HB;
 
     auto store_final = [&](int d, int h, int ps, int n, const float* v) {
       if (!kp.final_states || n >= g.N) return;
@@ -478,106 +604,105 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < kPT; c += 4)
         *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
     };
-    // output of tile (it-1): y = exp(cs) Yoff + Ydiag
-    auto emit_prev = [&](uint32_t pit) -> bool {
-      const uint32_t yb = pit & 1;
-      if (!wait_bar(bar(YDONE0 + yb), (pit >> 1) & 1, abort_flag, kp.status)) return false;
-      tc_fence_after();
-      const float sc = ex2(cs_s[(pit & 1) * 128 + r]);
-      const bool valid = r < prev_len;
-      __nv_bfloat16* dst = kp.y + ((prev_t0 + r) * g.H + prev_h) * (int64_t)g.P + prev_ps * kPT;
+    // documents without tokens: the final state is the initial state
+    for (int u = blockIdx.x; u < kp.units; u += gridDim.x) {
+      const Unit U = unit_of(kp, u);
+      if (U.ntiles != 0 || !kp.final_states) continue;
+      for (int mt = 0; mt < NT; ++mt) {
+        const int n = r + 128 * mt;
+        if (n >= g.N) continue;
+        float v[kPT];
+        const float* src =
+            kp.init ? kp.init + (((int64_t)U.d * g.H + U.h) * g.N + n) * g.P + U.ps * kPT : nullptr;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float yo[32], yd[32];
-        tc_ld32(tmem + lane_off + C::COL_YOFF + yb * kPT + half * 32, yo);
-        tc_ld32(tmem + lane_off + C::COL_YDIAG + yb * kPT + half * 32, yd);
-        tc_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint4 v;
-            v.x = pack_bf16(fmaf(sc, yo[c + 0], yd[c + 0]), fmaf(sc, yo[c + 1], yd[c + 1]));
-            v.y = pack_bf16(fmaf(sc, yo[c + 2], yd[c + 2]), fmaf(sc, yo[c + 3], yd[c + 3]));
-            v.z = pack_bf16(fmaf(sc, yo[c + 4], yd[c + 4]), fmaf(sc, yo[c + 5], yd[c + 5]));
-            v.w = pack_bf16(fmaf(sc, yo[c + 6], yd[c + 6]), fmaf(sc, yo[c + 7], yd[c + 7]));
-            *reinterpret_cast<uint4*>(dst + half * 32 + c) = v;
-          }
-        }
+        for (int c = 0; c < kPT; ++c) v[c] = src ? src[c] : 0.f;
+        store_final(U.d, U.h, U.ps, n, v);
       }
-      tc_fence_before();
-      mbar_arrive(bar(YFREE0 + yb));
-      return true;
+    }
+
+    // per-tile scalars, loaded one tile ahead
+    struct Pre {
+      float dt, A, bias, D;
+    };
+    auto prefetch = [&](const Cursor& c) -> Pre {
+      Pre p{0.f, 0.f, 0.f, 0.f};
+      if (!c.valid) return p;
+      const int len = min(kTile, c.U.len - c.jt * kTile);
+      if (r < len) p.dt = load_f(kp.dt, (c.U.start + (int64_t)c.jt * kTile + r) * g.H + c.U.h, 1);
+      p.A = kp.A[c.U.h];
+      p.bias = kp.dt_bias ? kp.dt_bias[c.U.h] : 0.f;
+      p.D = kp.D ? kp.D[c.U.h] : 0.f;
+      return p;
     };
 
-    for (int u = blockIdx.x; u < kp.units && ok; u += gridDim.x) {
-      const Unit U = unit_of(kp, u);
-      if (U.ntiles == 0) {  // empty document: the final state is the initial state
-        for (int mt = 0; mt < NT; ++mt) {
-          const int n = r + 128 * mt;
-          if (n >= g.N || !kp.final_states) continue;
-          float v[kPT];
-          const float* src = kp.init ? kp.init + (((int64_t)U.d * g.H + U.h) * g.N + n) * g.P + U.ps * kPT
-                                     : nullptr;
-#pragma unroll
-          for (int c = 0; c < kPT; ++c) v[c] = src ? src[c] : 0.f;
-          store_final(U.d, U.h, U.ps, n, v);
-        }
-        continue;
-      }
-      const float Ah = kp.A[U.h];
-      const float bias = kp.dt_bias ? kp.dt_bias[U.h] : 0.f;
-      const float Dh = kp.D ? kp.D[U.h] : 0.f;
-      for (int jt = 0; jt < U.ntiles && ok; ++jt, ++it) {
-        const int64_t t0 = U.start + (int64_t)jt * kTile;
-        const int len = min(kTile, U.len - jt * kTile);
-        const uint32_t s = it % C::NSTAGE, k = it / C::NSTAGE;
-        const uint32_t cb = (it & 1) * 128;
-        // ---- E1: delta and in-tile cumulative log decay (scaled by log2 e) ----
-        float dl = 0.f, la = 0.f;
-        if (r < len) {
-          const float z = load_f(kp.dt, (t0 + r) * g.H + U.h, 1) + bias;
-          dl = softplus_f(z);
-          la = dl * Ah * LOG2E;
-        }
-        float v = la;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float t = __shfl_up_sync(0xffffffffu, v, o);
-          if (lane >= o) v += t;
-        }
-        epi_sync();  // previous readers of wsum / cs slot are done
-        if (lane == 31) wsum[q] = v;
-        epi_sync();
-        for (int w = 0; w < q; ++w) v += wsum[w];
-        cs_s[cb + r] = v;
-        dl_s[cb + r] = dl;
-        epi_sync();
-        const float cs_last = cs_s[cb + 127];
-        const float cs_r = v;
+    uint32_t it = 0;
+    bool ok = true;
+    bool pend = false;
+    int pend_d = 0, pend_h = 0, pend_ps = 0;
+    Cursor cur = cursor_first(kp);
+    Cursor nxt = cur;
+    cursor_next(kp, nxt);
+    Pre pc = prefetch(cur);
+    for (; cur.valid && ok; ++it) {
+      const Unit& U = cur.U;
+      const int jt = cur.jt;
+      const int len = min(kTile, U.len - jt * kTile);
+      const uint32_t cb = (it & 1) * 128;
+      const Pre pn = prefetch(nxt);  // consumed one tile later
 
-        // ---- E3: state entering the tile -> bf16 copy (Hb), decayed copy in TMEM ----
-        if (it > 0) ok = wait_bar(bar(STATE_DONE), (it - 1) & 1, abort_flag, kp.status);
-        if (!ok) break;
-        tc_fence_after();
-        const float decay = ex2(cs_last);
+      // ---- E1: delta and in-tile cumulative log decay (scaled by log2 e) ----
+      float dl = 0.f, la = 0.f;
+      if (r < len) {
+        dl = softplus_f(pc.dt + pc.bias);
+        la = dl * pc.A * LOG2E;
+      }
+      float cs = la;
 #pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float t = __shfl_up_sync(0xffffffffu, cs, o);
+        if (lane >= o) cs += t;
+      }
+      float* ws = wsum + (it & 1) * 4;
+      if (lane == 31) ws[q] = cs;
+      // the cs buffer of this parity was last read by epilogue B two tiles ago
+      if (it >= 2) ok = wait_bar(bar(CS_FREE0 + (it & 1)), ((it - 2) >> 1) & 1, abort_flag, kp.status);
+      sync_a();
+      if (!ok) break;
+      for (int w = 0; w < q; ++w) cs += ws[w];
+      const float cs_last = ws[0] + ws[1] + ws[2] + ws[3];
+      const float cs_blockend = __shfl_sync(0xffffffffu, cs, 31);
+      cs_s[cb + r] = cs;
+      dl_s[cb + r] = dl;
+      v_s[cb + r] = ex2(cs_blockend - cs) * dl;
+      w_s[cb + r] = ex2(cs_last - cs) * dl;
+      mbar_arrive(bar(CS_READY0 + (it & 1)));
+
+      // ---- E3: state entering the tile -> bf16 copy Hb; decayed copy stays in TMEM ----
+      if (it > 0) ok = wait_bar(bar(STATE_DONE), (it - 1) & 1, abort_flag, kp.status);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const float decay = ex2(cs_last);
+        const uint32_t hb_base = hb0 + (C::HB_BUFS == 2 ? (it & 1) : 0) * C::HB_BYTES;
+#pragma unroll 1
         for (int mt = 0; mt < NT; ++mt) {
           const int n = r + 128 * mt;
           const uint32_t th = tmem + lane_off + C::COL_H + mt * kPT;
           float hv[kPT];
           if (jt == 0) {
-            if (pend) {
+            if (pend) {  // the previous unit's final state is still in TMEM
               tc_ld32(th, hv);
               tc_ld32(th + 32, hv + 32);
               tc_wait_ld();
               store_final(pend_d, pend_h, pend_ps, n, hv);
             }
-            const float* src = (kp.init && n < g.N)
-                                   ? kp.init + (((int64_t)U.d * g.H + U.h) * g.N + n) * g.P + U.ps * kPT
-                                   : nullptr;
+            const float* src =
+                (kp.init && n < g.N)
+                    ? kp.init + (((int64_t)U.d * g.H + U.h) * g.N + n) * g.P + U.ps * kPT
+                    : nullptr;
 #pragma unroll
             for (int c = 0; c < kPT; c += 4) {
-              float4 f = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0, 0, 0, 0);
+              const float4 f = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0, 0, 0, 0);
               hv[c] = f.x;
               hv[c + 1] = f.y;
               hv[c + 2] = f.z;
@@ -588,13 +713,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_ld32(th + 32, hv + 32);
             tc_wait_ld();
           }
-          // Hb row n (MN-major operand of Yoff: rows = n, 128 bytes of p per row)
+          // Hb row n: the MN-major B operand of Yoff (rows = n, 128 bytes of p)
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            st_shared_v4(hb_base + swz((uint32_t)n, (uint32_t)c),
-                         pack_bf16(hv[8 * c + 0], hv[8 * c + 1]), pack_bf16(hv[8 * c + 2], hv[8 * c + 3]),
-                         pack_bf16(hv[8 * c + 4], hv[8 * c + 5]), pack_bf16(hv[8 * c + 6], hv[8 * c + 7]));
-          }
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(hb_base + swz((uint32_t)n, (uint32_t)c), pack_bf16(hv[8 * c], hv[8 * c + 1]),
+                         pack_bf16(hv[8 * c + 2], hv[8 * c + 3]), pack_bf16(hv[8 * c + 4], hv[8 * c + 5]),
+                         pack_bf16(hv[8 * c + 6], hv[8 * c + 7]));
 #pragma unroll
           for (int c = 0; c < kPT; ++c) hv[c] *= decay;
           tc_st32(th, hv);
@@ -602,90 +726,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         pend = false;
         tc_wait_st();
-
-        // ---- E4: XW = w o x_j,  w_s = exp(cs_last - cs_s) delta_s ----
-        ok = wait_bar(bar(FULL0 + s), k & 1, abort_flag, kp.status);
-        if (!ok) break;
-        {
-          const float wr = ex2(cs_last - cs_r) * dl;
-          const uint32_t xrow = sbase + s * C::STAGE_BYTES;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 xv = ld_shared_v4(xrow + swz((uint32_t)r, (uint32_t)c));
-            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
-            float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
-            float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
-            st_shared_v4(xw_base + swz((uint32_t)r, (uint32_t)c), pack_bf16(wr * f0.x, wr * f0.y),
-                         pack_bf16(wr * f1.x, wr * f1.y), pack_bf16(wr * f2.x, wr * f2.y),
-                         pack_bf16(wr * f3.x, wr * f3.y));
-          }
-        }
         fence_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(PREP));
-
-        // ---- E2: decay mask of the diagonal block -> M (bf16, K-major) ----
-        ok = wait_bar(bar(CB_DONE), it & 1, abort_flag, kp.status);
-        if (ok && it > 0) ok = wait_bar(bar(YDONE0 + ((it - 1) & 1)), ((it - 1) >> 1) & 1, abort_flag,
-                                        kp.status);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const uint32_t panel = m_base + (uint32_t)(cc >> 1) * kPanel;
-          if (cc > q) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              st_shared_v4(panel + swz((uint32_t)r, (uint32_t)((cc & 1) * 4 + i)), 0u, 0u, 0u, 0u);
-            continue;
-          }
-          float zv[32];
-          tc_ld32(tmem + lane_off + C::COL_Z + cc * 32, zv);
-          tc_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int sidx = cc * 32 + j;
-            float m = zv[j] * ex2(cs_r - cs_s[cb + sidx]) * dl_s[cb + sidx];
-            if (sidx == r) m += Dh;
-            zv[j] = sidx <= r ? m : 0.f;
-          }
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            st_shared_v4(panel + swz((uint32_t)r, (uint32_t)((cc & 1) * 4 + i)),
-                         pack_bf16(zv[8 * i + 0], zv[8 * i + 1]), pack_bf16(zv[8 * i + 2], zv[8 * i + 3]),
-                         pack_bf16(zv[8 * i + 4], zv[8 * i + 5]), pack_bf16(zv[8 * i + 6], zv[8 * i + 7]));
-        }
-        tc_fence_before();
-        mbar_arrive(bar(Z_FREE));
-        fence_async_smem();
-        mbar_arrive(bar(M_READY));
-
-        // ---- E5 of the previous tile ----
-        if (prev) {
-          if (!emit_prev(it - 1)) {
-            ok = false;
-            break;
-          }
-        }
-        prev = true;
-        prev_t0 = t0;
-        prev_len = len;
-        prev_h = U.h;
-        prev_ps = U.ps;
-        if (jt == U.ntiles - 1) {
-          pend = true;
-          pend_d = U.d;
-          pend_h = U.h;
-          pend_ps = U.ps;
-        }
+        mbar_arrive(bar(HB_READY));
       }
+
+      // ---- E2 (blocks 0 and q; the rest of the causal part is epilogue B's) ----
+      ok = wait_bar(bar(CB_DONE0 + (it & 1)), (it >> 1) & 1, abort_flag, kp.status);
+      if (ok) ok = wait_bar(bar(CS_READY0 + (it & 1)), (it >> 1) & 1, abort_flag, kp.status);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const uint32_t zaddr = tmem + lane_off + C::COL_Z + (it & 1) * 128;
+        mask_block(zaddr, 0, q, r, cs, cs_s + cb, dl_s + cb, v_s + cb, pc.D);
+        if (q > 0) mask_block(zaddr, q, q, r, cs, cs_s + cb, dl_s + cb, v_s + cb, pc.D);
+#pragma unroll 1
+        for (int cc = q + 1; cc < 4; ++cc) zero_block(zaddr, cc);
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(M_READY_A0 + (it & 1)));
+      }
+
+      if (jt == U.ntiles - 1) {
+        pend = true;
+        pend_d = U.d;
+        pend_h = U.h;
+        pend_ps = U.ps;
+      }
+      cur = nxt;
+      cursor_next(kp, nxt);
+      pc = pn;
     }
-    if (ok && prev) ok = emit_prev(it - 1);
     if (ok && pend) {
       ok = wait_bar(bar(STATE_DONE), (it - 1) & 1, abort_flag, kp.status);
       if (ok) {
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int mt = 0; mt < NT; ++mt) {
           float hv[kPT];
           const uint32_t th = tmem + lane_off + C::COL_H + mt * kPT;
@@ -696,6 +772,107 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+  } else {
+    // ========= epilogue B: weighted input, mask blocks 1..q-1, outputs =========
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t xw_base = sbase + C::OFF_XW;
+    uint32_t it = 0;
+    bool ok = true;
+    bool prev = false;
+    int64_t prev_t0 = 0;
+    int prev_len = 0, prev_h = 0, prev_ps = 0;
+    float prev_el = 0.f;
+
+    // output of tile pit: y = exp(cs) Yoff + Ydiag
+    auto emit = [&](uint32_t pit) -> bool {
+      if (!wait_bar(bar(YDONE0 + (pit & 1)), (pit >> 1) & 1, abort_flag, kp.status)) return false;
+      tc_fence_after();
+      const bool valid = r < prev_len;
+      __nv_bfloat16* dst = kp.y + ((prev_t0 + r) * g.H + prev_h) * (int64_t)g.P + prev_ps * kPT;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        float yo[32], yd[32];
+        tc_ld32(tmem + lane_off + C::COL_YOFF + half * 32, yo);
+        tc_ld32(tmem + lane_off + C::COL_YDIAG + half * 32, yd);
+        tc_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint4 v;
+            v.x = pack_bf16(fmaf(prev_el, yo[c + 0], yd[c + 0]), fmaf(prev_el, yo[c + 1], yd[c + 1]));
+            v.y = pack_bf16(fmaf(prev_el, yo[c + 2], yd[c + 2]), fmaf(prev_el, yo[c + 3], yd[c + 3]));
+            v.z = pack_bf16(fmaf(prev_el, yo[c + 4], yd[c + 4]), fmaf(prev_el, yo[c + 5], yd[c + 5]));
+            v.w = pack_bf16(fmaf(prev_el, yo[c + 6], yd[c + 6]), fmaf(prev_el, yo[c + 7], yd[c + 7]));
+            *reinterpret_cast<uint4*>(dst + half * 32 + c) = v;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(Y_FREE));
+      return true;
+    };
+
+    for (Cursor c = cursor_first(kp); c.valid && ok; cursor_next(kp, c), ++it) {
+      const uint32_t s = it % C::NSTAGE, k = it / C::NSTAGE, cb = (it & 1) * 128;
+      // the four warps of this group finish a tile (and all its barrier arrivals)
+      // before any of them starts the next, so arrivals never mix tiles
+      sync_b();
+      // ---- E4: XW = w o x_j ----
+      ok = wait_bar(bar(CS_READY0 + (it & 1)), (it >> 1) & 1, abort_flag, kp.status);
+      if (!ok) break;
+      const float wr = w_s[cb + r];
+      const float cs_r = cs_s[cb + r];
+      const float el = ex2(cs_r);
+      ok = wait_bar(bar(FULL0 + s), k & 1, abort_flag, kp.status);
+      // XW is free once the previous tile's state update has read it
+      if (ok && it > 0) ok = wait_bar(bar(STATE_DONE), (it - 1) & 1, abort_flag, kp.status);
+      if (!ok) break;
+      {
+        const uint32_t xrow = sbase + s * C::STAGE_BYTES;
+#pragma unroll
+        for (int cidx = 0; cidx < 8; ++cidx) {
+          const uint4 xv = ld_shared_v4(xrow + swz((uint32_t)r, (uint32_t)cidx));
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+          const float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
+          const float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
+          st_shared_v4(xw_base + swz((uint32_t)r, (uint32_t)cidx), pack_bf16(wr * f0.x, wr * f0.y),
+                       pack_bf16(wr * f1.x, wr * f1.y), pack_bf16(wr * f2.x, wr * f2.y),
+                       pack_bf16(wr * f3.x, wr * f3.y));
+        }
+      }
+      fence_async_smem();
+      mbar_arrive(bar(XW_READY));
+
+      // ---- E2 (off-diagonal blocks 1..q-1 of this lane quarter) ----
+      ok = wait_bar(bar(CB_DONE0 + (it & 1)), (it >> 1) & 1, abort_flag, kp.status);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const uint32_t zaddr = tmem + lane_off + C::COL_Z + (it & 1) * 128;
+#pragma unroll 1
+        for (int cc = 1; cc < q; ++cc)
+          mask_block(zaddr, cc, q, r, cs_r, cs_s + cb, dl_s + cb, v_s + cb, 0.f);
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(M_READY_B0 + (it & 1)));
+      }
+      mbar_arrive(bar(CS_FREE0 + (it & 1)));  // done with this tile's cs buffer
+
+      // ---- E5 of the previous tile ----
+      if (prev && !emit(it - 1)) {
+        ok = false;
+        break;
+      }
+      prev = true;
+      prev_t0 = c.U.start + (int64_t)c.jt * kTile;
+      prev_len = min(kTile, c.U.len - c.jt * kTile);
+      prev_h = c.U.h;
+      prev_ps = c.U.ps;
+      prev_el = el;
+    }
+    if (ok && prev) emit(it - 1);
   }
 
   // ---- teardown ----
