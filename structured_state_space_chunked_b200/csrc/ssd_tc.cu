@@ -45,7 +45,7 @@ namespace {
 
 constexpr int kTile = 128;          // tokens per tile
 constexpr int kPT = 64;             // head-dim columns per unit
-constexpr int kThreads = 320;       // 10 warps: TMA, MMA, epilogue A (4), epilogue B (4)
+constexpr int kThreads = 320;       // 10 warps: MMA, TMA, two epilogue groups of 4
 constexpr uint32_t kPanel = 16384;  // one 128-row x 128-byte SW128 panel
 
 template <int NT>
@@ -58,20 +58,18 @@ struct Cfg {
   static constexpr uint32_t BC_BYTES = NPANEL * kPanel;
   static constexpr uint32_t STAGE_BYTES = X_BYTES + 2 * BC_BYTES;
   static constexpr uint32_t HB_BYTES = NPAD * 128;
-  static constexpr uint32_t OFF_XW = NSTAGE * STAGE_BYTES;
-  static constexpr uint32_t OFF_HB = OFF_XW + kPanel;
+  static constexpr uint32_t OFF_XW = NSTAGE * STAGE_BYTES;         // [2] one per epilogue group
+  static constexpr uint32_t OFF_HB = OFF_XW + 2 * kPanel;          // [HB_BUFS]
   static constexpr uint32_t OFF_SMALL = OFF_HB + HB_BUFS * HB_BYTES;
-  static constexpr uint32_t OFF_CS = OFF_SMALL;       // float[2][128]  cs * log2(e)
-  static constexpr uint32_t OFF_DL = OFF_CS + 1024;   // float[2][128]  delta
-  static constexpr uint32_t OFF_V = OFF_DL + 1024;    // float[2][128]  exp(cs_blockend - cs) delta
-  static constexpr uint32_t OFF_W = OFF_V + 1024;     // float[2][128]  exp(cs_last - cs) delta
-  static constexpr uint32_t OFF_WS = OFF_W + 1024;    // scan scratch [2][4] and flags
+  static constexpr uint32_t OFF_V = OFF_SMALL;        // float[2][128] exp(cs_blockend - cs) delta
+  static constexpr uint32_t OFF_WS = OFF_V + 1024;    // float[2][4] scan totals, then flags
   static constexpr uint32_t OFF_BAR = OFF_WS + 64;    // mbarriers
   static constexpr uint32_t OFF_TMEM = OFF_BAR + 256;
-  static constexpr uint32_t SMEM = OFF_TMEM + 64;
-  // TMEM columns: two C B^T tiles (each turned in place into the bf16 mask
-  // operand M), the two output accumulators and the state (NT lane tiles)
-  static constexpr uint32_t COL_Z = 0, COL_YOFF = 256, COL_YDIAG = 320, COL_H = 384;
+  static constexpr uint32_t SMEM = OFF_TMEM + 16;
+  // TMEM columns: per epilogue group a 128-column C B^T tile, turned in place into
+  // the bf16 mask operand M (columns 0..63) with Ydiag accumulated next to it
+  // (columns 64..127); per group a Yoff accumulator; the state
+  static constexpr uint32_t COL_Z = 0, COL_Y = 256, COL_H = 384;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t TX_BYTES = X_BYTES + 2 * BC_BYTES;
 };
@@ -79,9 +77,16 @@ static_assert(Cfg<1>::SMEM <= 232448, "smem budget");
 static_assert(Cfg<2>::SMEM <= 232448, "smem budget");
 static_assert(Cfg<2>::COL_H + 64 * 2 <= 512, "tmem budget");
 
+// Barriers.  Index +w is epilogue group w (tiles it with it % 2 == w).
 enum Bar {
-  FULL0 = 0, FULL1, EMPTY0, EMPTY1, CB_DONE0, CB_DONE1, STATE_DONE, HB_READY, XW_READY,
-  M_READY_A0, M_READY_A1, M_READY_B0, M_READY_B1, YDONE0, YDONE1, Y_FREE, CS_READY0, CS_READY1, CS_FREE0, CS_FREE1,
+  FULL0 = 0, FULL1, EMPTY0, EMPTY1,
+  CB_DONE0, CB_DONE1,       // C B^T of the group's tile is in its Z buffer (MMA -> group)
+  M_READY0, M_READY1,       // mask operand written over Z (group -> MMA)
+  Z_FREE0, Z_FREE1,         // the group has read Ydiag from its Z buffer (group -> MMA)
+  XW_READY0, XW_READY1,     // w o x written (group -> MMA)
+  PREP0, PREP1,             // state decayed in TMEM, Hb written, Ydiag read (group -> MMA)
+  STATE_DONE0, STATE_DONE1, // state update of the group's tile done (MMA -> other group)
+  YO_DONE0, YO_DONE1,       // Ydiag and Yoff done (MMA -> group; other group if one Hb)
   TEARDOWN, NBAR
 };
 
@@ -296,7 +301,7 @@ struct Cursor {
   bool valid;
   Unit U;
 };
-__device__ __forceinline__ void cursor_next(const KParams& kp, Cursor& c) {
+__device__ __noinline__ void cursor_next(const KParams& kp, Cursor& c) {
   if (c.valid && c.jt + 1 < c.U.ntiles) {
     ++c.jt;
     return;
@@ -322,9 +327,8 @@ __device__ __forceinline__ Cursor cursor_first(const KParams& kp) {
 
 // Bounded wait: false (and the abort flag raised) if the phase did not complete
 // within ~2 s or another role already gave up.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         int* status) {
-  if (mbar_try(bar, parity)) return true;
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity,
+                                           volatile int* abort_flag, int* status) {
   const uint64_t t0 = globaltimer();
   uint32_t n = 0;
   while (!mbar_try(bar, parity)) {
@@ -339,42 +343,140 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
   return true;
 }
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int* status) {
+  return mbar_try(bar, parity) || wait_bar_slow(bar, parity, abort_flag, status);
+}
 
-// Decay mask of column block cc (s in [32cc, 32cc+32)) for this thread's row r of
-// the diagonal block: reads C B^T from TMEM (Z) and writes M[r, s] as bf16 pairs
-// into the first 16 columns of the same 32-column block (in place, so any warp of
-// the lane quarter may handle any block).  Blocks left of the diagonal block use
-// exp(cs_r - cs_s) = exp(cs_r - cs_b) exp(cs_b - cs_s), b = 32cc + 31, with the
-// second factor (times delta_s) precomputed per column in v.
-__device__ __forceinline__ void mask_block(uint32_t zaddr, int cc, int q, int r, float cs_r,
-                                           const float* cs, const float* dl, const float* v,
-                                           float Dh) {
+// Final state row n (64 columns of the unit's P slice) from TMEM to final_states.
+__device__ __noinline__ void tmem_state_to_final(const KParams& kp, uint32_t th, int d, int h,
+                                                 int ps, int n) {
+  float hv[kPT];
+  tc_ld32(th, hv);
+  tc_ld32(th + 32, hv + 32);
+  tc_wait_ld();
+  if (!kp.final_states || n >= kp.g.N) return;
+  float* dst = kp.final_states + (((int64_t)d * kp.g.H + h) * kp.g.N + n) * kp.g.P + ps * kPT;
+#pragma unroll
+  for (int c = 0; c < kPT; c += 4)
+    *reinterpret_cast<float4*>(dst + c) = make_float4(hv[c], hv[c + 1], hv[c + 2], hv[c + 3]);
+}
+
+// State row n on entry to a unit's first tile: the initial state (or zero) goes
+// to Hb as bf16 and, decayed by the tile, into TMEM for the state update.
+__device__ __noinline__ void enter_unit_row(const KParams& kp, uint32_t th, uint32_t hb_base,
+                                            int d, int h, int ps, int n, float decay) {
+  const float* src = (kp.init && n < kp.g.N)
+                         ? kp.init + (((int64_t)d * kp.g.H + h) * kp.g.N + n) * kp.g.P + ps * kPT
+                         : nullptr;
+  float hv[kPT];
+#pragma unroll
+  for (int c = 0; c < kPT; c += 4) {
+    const float4 f = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0, 0, 0, 0);
+    hv[c] = f.x;
+    hv[c + 1] = f.y;
+    hv[c + 2] = f.z;
+    hv[c + 3] = f.w;
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    st_shared_v4(hb_base + swz((uint32_t)n, (uint32_t)c), pack_bf16(hv[8 * c], hv[8 * c + 1]),
+                 pack_bf16(hv[8 * c + 2], hv[8 * c + 3]), pack_bf16(hv[8 * c + 4], hv[8 * c + 5]),
+                 pack_bf16(hv[8 * c + 6], hv[8 * c + 7]));
+#pragma unroll
+  for (int c = 0; c < kPT; ++c) hv[c] *= decay;
+  tc_st32(th, hv);
+  tc_st32(th + 32, hv + 32);
+}
+
+// Documents without tokens: their final state is their initial state (or zero).
+__device__ __noinline__ void empty_units_final(const KParams& kp, int r, int nt) {
+  if (!kp.final_states) return;
+  for (int u = blockIdx.x; u < kp.units; u += gridDim.x) {
+    const Unit U = unit_of(kp, u);
+    if (U.ntiles != 0) continue;
+    for (int mt = 0; mt < nt; ++mt) {
+      const int n = r + 128 * mt;
+      if (n >= kp.g.N) continue;
+      const int64_t off = (((int64_t)U.d * kp.g.H + U.h) * kp.g.N + n) * kp.g.P + U.ps * kPT;
+      for (int c = 0; c < kPT; ++c) kp.final_states[off + c] = kp.init ? kp.init[off + c] : 0.f;
+    }
+  }
+}
+
+// Off-diagonal column block cc (< q) of the diagonal tile for this thread's row:
+// M[r, s] = Z[r, s] exp(cs_r - cs_b) v[s],  b = 32cc + 31,  v[s] = exp(cs_b - cs_s) delta_s
+// (the decay factorises across the block boundary and both factors are <= 1).
+// Reads C B^T from TMEM and writes M as bf16 pairs to columns 16cc..16cc+15 (in
+// place: a warp handles its blocks in increasing cc, so the columns written were
+// already read).
+__device__ __noinline__ void mask_off(uint32_t zaddr, int cc, float cs_r, float cs_b,
+                                      const float* v) {
   float zv[32];
   tc_ld32(zaddr + 32 * cc, zv);
   tc_wait_ld();
-  if (cc < q) {
-    const float u = ex2(cs_r - cs[32 * cc + 31]);
+  const float u = ex2(cs_r - cs_b);
+  uint32_t pk[16];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) zv[j] *= u * v[32 * cc + j];
-  } else {
+  for (int i = 0; i < 16; ++i)
+    pk[i] = pack_bf16(zv[2 * i] * (u * v[32 * cc + 2 * i]), zv[2 * i + 1] * (u * v[32 * cc + 2 * i + 1]));
+  tc_st16(zaddr + 16 * cc, pk);
+}
+// Diagonal 32 x 32 block of warp q: rows and columns both belong to this warp's
+// lanes, so cs_s and delta_s come from the lanes by shuffle.  M[r, s] =
+// Z exp(cs_r - cs_s) delta_s for s <= r, 0 above; the skip term D sits on s = r.
+__device__ __noinline__ void mask_diag(uint32_t zaddr, int q, int lane, float cs, float dl,
+                                       float Dh) {
+  float zv[32];
+  tc_ld32(zaddr + 32 * q, zv);
+  tc_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int sidx = 32 * cc + j;
-      float m = zv[j] * ex2(cs_r - cs[sidx]) * dl[sidx];
-      if (sidx == r) m += Dh;
-      zv[j] = sidx <= r ? m : 0.f;
-    }
+  for (int j = 0; j < 32; ++j) {
+    const float cj = __shfl_sync(0xffffffffu, cs, j);
+    const float dj = __shfl_sync(0xffffffffu, dl, j);
+    float m = zv[j] * ex2(cs - cj) * dj;
+    if (j == lane) m += Dh;
+    zv[j] = j <= lane ? m : 0.f;
   }
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(zv[2 * i], zv[2 * i + 1]);
-  tc_st16(zaddr + 32 * cc, pk);
+  tc_st16(zaddr + 16 * q, pk);
 }
 __device__ __forceinline__ void zero_block(uint32_t zaddr, int cc) {
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) pk[i] = 0u;
-  tc_st16(zaddr + 32 * cc, pk);
+  tc_st16(zaddr + 16 * cc, pk);
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(a), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Number of tiles this CTA processes, and the last unit of its stream with tokens.
+__device__ __noinline__ uint32_t count_tiles(const KParams& kp, int* last_unit) {
+  uint32_t n = 0;
+  *last_unit = -1;
+  for (int u = blockIdx.x; u < kp.units; u += gridDim.x) {
+    const Unit U = unit_of(kp, u);
+    n += (uint32_t)U.ntiles;
+    if (U.ntiles > 0) *last_unit = u;
+  }
+  return n;
+}
+// The unit with tokens that precedes unit u in this CTA's stream.
+__device__ __noinline__ int prev_unit_with_tiles(const KParams& kp, int u) {
+  for (u -= gridDim.x; u >= 0; u -= gridDim.x)
+    if (unit_of(kp, u).ntiles > 0) return u;
+  return -1;
 }
 
 template <int NT>
@@ -385,11 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = su32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* cs_s = reinterpret_cast<float*>(smem + C::OFF_CS);
-  float* dl_s = reinterpret_cast<float*>(smem + C::OFF_DL);
-  float* v_s = reinterpret_cast<float*>(smem + C::OFF_V);
-  float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
-  float* wsum = reinterpret_cast<float*>(smem + C::OFF_WS);
+  float* v_all = reinterpret_cast<float*>(smem + C::OFF_V);
+  float* ws_all = reinterpret_cast<float*>(smem + C::OFF_WS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_WS + 32);
   int* bad_flag = reinterpret_cast<int*>(smem + C::OFF_WS + 36);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
@@ -419,30 +518,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   if (threadIdx.x == 0) {
-    mbar_init(bar(FULL0), 1);
-    mbar_init(bar(FULL1), 1);
-    mbar_init(bar(EMPTY0), 1);
-    mbar_init(bar(EMPTY1), 1);
-    mbar_init(bar(CB_DONE0), 1);
-    mbar_init(bar(CB_DONE1), 1);
-    mbar_init(bar(STATE_DONE), 1);
-    mbar_init(bar(HB_READY), 128);
-    mbar_init(bar(XW_READY), 128);
-    mbar_init(bar(M_READY_A0), 128);
-    mbar_init(bar(M_READY_A1), 128);
-    mbar_init(bar(M_READY_B0), 128);
-    mbar_init(bar(M_READY_B1), 128);
-    mbar_init(bar(YDONE0), 1);
-    mbar_init(bar(YDONE1), 1);
-    mbar_init(bar(Y_FREE), 128);
-    mbar_init(bar(CS_READY0), 128);
-    mbar_init(bar(CS_READY1), 128);
-    mbar_init(bar(CS_FREE0), 128);
-    mbar_init(bar(CS_FREE1), 128);
-    mbar_init(bar(TEARDOWN), 1);
+    for (int i = 0; i < NBAR; ++i) {
+      const bool group = i == M_READY0 || i == M_READY1 || i == XW_READY0 || i == XW_READY1 ||
+                         i == PREP0 || i == PREP1 || i == Z_FREE0 || i == Z_FREE1;
+      mbar_init(bar(i), group ? 128 : 1);
+    }
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      su32(tmem_slot)),
                  "r"(C::TMEM_COLS)
@@ -453,8 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  int last_unit = -1;
+  const uint32_t ntiles = count_tiles(kp, &last_unit);
 
-  if (warp == 0) {
+  if (warp == 1) {
     // ================================ TMA producer ================================
     if (lane == 0) {
       uint32_t it = 0;
@@ -484,143 +569,134 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 0) {
     // ================================ MMA issuer =================================
+    // Event loop over three in-order streams of work: C B^T (at most two tiles ahead
+    // of Ydiag, one per Z buffer), Ydiag (after the group's mask), and the state
+    // update + left factors (after the group's state hand-over).  Readiness is
+    // polled without blocking so that whichever group is ready is served first.
     if (lane == 0) {
       constexpr uint32_t ID_CB = idesc(128, 128, 0, 0);    // Z = C B^T, both K-major
       constexpr uint32_t ID_YOFF = idesc(128, kPT, 0, 1);  // Yoff = C Hb, Hb MN-major
       constexpr uint32_t ID_ST = idesc(128, kPT, 1, 1);    // H += B^T XW, both MN-major
       constexpr uint32_t ID_YD = idesc(128, kPT, 0, 1);    // Ydiag = M X, M in TMEM, X MN-major
-      // with two stages, C B^T of the next tile is issued before this tile's mask is
-      // ready, so the tensor cores work while the epilogue builds M
-      constexpr bool LOOKAHEAD = C::NSTAGE >= 2;
-      const uint32_t xw_base = sbase + C::OFF_XW, hb0 = sbase + C::OFF_HB;
-      auto stage_of = [&](uint32_t i) { return sbase + (i % C::NSTAGE) * C::STAGE_BYTES; };
-      // Z = C_j B_j^T for tile i (waits for its data and for its Z buffer)
-      auto issue_cb = [&](uint32_t i) -> bool {
-        const uint32_t st = stage_of(i), zb = i & 1;
-        if (!wait_bar(bar(FULL0 + i % C::NSTAGE), (i / C::NSTAGE) & 1, abort_flag, kp.status))
-          return false;
-        // Z buffer zb last held the mask operand of tile i-2
-        if (i >= 2 && !wait_bar(bar(YDONE0 + zb), ((i - 2) >> 1) & 1, abort_flag, kp.status))
-          return false;
-        tc_fence_after();
-        const uint32_t b_base = st + C::X_BYTES, c_base = st + C::X_BYTES + C::BC_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < C::NPAD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-          tc_mma(tmem + C::COL_Z + zb * 128, sdesc(c_base + off, 16, 1024),
-                 sdesc(b_base + off, 16, 1024), ID_CB, kk > 0);
-        }
-        tc_commit(bar(CB_DONE0 + zb));
-        return true;
-      };
-      uint32_t it = 0;
-      bool ok = true;
-      Cursor c = cursor_first(kp);
-      if (c.valid && LOOKAHEAD) ok = issue_cb(0);
-      for (; c.valid && ok; ++it) {
-        Cursor n = c;
-        cursor_next(kp, n);
-        const uint32_t s = it % C::NSTAGE, zb = it & 1;
-        const uint32_t st = stage_of(it);
-        const uint32_t x_base = st, b_base = st + C::X_BYTES, c_base = st + C::X_BYTES + C::BC_BYTES;
-        const uint32_t hb_base = hb0 + (C::HB_BUFS == 2 ? zb : 0) * C::HB_BYTES;
-        if (!LOOKAHEAD && !(ok = issue_cb(it))) break;
-        ok = wait_bar(bar(HB_READY), it & 1, abort_flag, kp.status);
-        if (ok) ok = wait_bar(bar(XW_READY), it & 1, abort_flag, kp.status);
-        if (!ok) break;
-        tc_fence_after();
-        auto issue_state = [&]() {
-          // H += B_j^T XW : K = tokens; A = the B tile read MN-major (n), B = XW MN-major (p)
-#pragma unroll
-          for (int mt = 0; mt < NT; ++mt)
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk)
-              tc_mma(tmem + C::COL_H + mt * kPT,
-                     sdesc(b_base + 2 * mt * kPanel + kk * 2048, kPanel, 1024),
-                     sdesc(xw_base + kk * 2048, kPanel, 1024), ID_ST, 1);
-        };
-        auto issue_yoff = [&]() {
-          // Yoff = C_j Hb : K = state dim; Hb rows are n (K), 128 bytes of p (MN)
+      auto stage = [&](uint32_t i) { return sbase + (i % C::NSTAGE) * C::STAGE_BYTES; };
+      uint32_t ncb = 0, nyd = 0, nst = 0;
+      uint64_t t_last = globaltimer();
+      uint32_t idle = 0;
+      while (nst < ntiles) {
+        bool did = false;
+        if (ncb < ntiles && ncb < nyd + 2 &&
+            mbar_test(bar(FULL0 + ncb % C::NSTAGE), (ncb / C::NSTAGE) & 1) &&
+            (ncb < 2 || mbar_test(bar(Z_FREE0 + (ncb & 1)), ((ncb - 2) >> 1) & 1))) {
+          // Z[w] = C_j B_j^T : K = state dim
+          tc_fence_after();
+          const uint32_t st = stage(ncb), w = ncb & 1;
+          const uint64_t dc = sdesc(st + C::X_BYTES + C::BC_BYTES, 16, 1024);
+          const uint64_t db = sdesc(st + C::X_BYTES, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < C::NPAD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kPanel + (kk & 3) * 32;
-            tc_mma(tmem + C::COL_YOFF, sdesc(c_base + off, 16, 1024),
-                   sdesc(hb_base + kk * 2048, C::HB_BYTES, 1024), ID_YOFF, kk > 0);
+            const uint64_t off = ((kk >> 2) * kPanel + (kk & 3) * 32) >> 4;
+            tc_mma(tmem + C::COL_Z + w * 128, dc + off, db + off, ID_CB, kk > 0);
           }
-        };
-        if (C::HB_BUFS == 2) {
-          issue_state();
-          tc_commit(bar(STATE_DONE));
-          if (LOOKAHEAD && n.valid && !(ok = issue_cb(it + 1))) break;
-          if (it >= 1) ok = wait_bar(bar(Y_FREE), (it - 1) & 1, abort_flag, kp.status);
-          if (!ok) break;
+          tc_commit(bar(CB_DONE0 + w));
+          ++ncb;
+          did = true;
+        } else if (nyd < ncb && mbar_test(bar(M_READY0 + (nyd & 1)), (nyd >> 1) & 1)) {
+          // Ydiag = M X_j : K = tokens.  M sits in TMEM as bf16 pairs (the 16 tokens of
+          // K step kk in columns 8kk..8kk+7 of the Z buffer); Ydiag goes next to it
           tc_fence_after();
-          issue_yoff();
-        } else {
-          // one Hb buffer: Yoff must have read it before the next state copy lands
-          if (it >= 1) ok = wait_bar(bar(Y_FREE), (it - 1) & 1, abort_flag, kp.status);
-          if (!ok) break;
-          tc_fence_after();
-          issue_yoff();
-          issue_state();
-          tc_commit(bar(STATE_DONE));
-          if (LOOKAHEAD && n.valid && !(ok = issue_cb(it + 1))) break;
-        }
-        // one barrier per tile parity and group: with C B^T issued a tile ahead, a
-        // group may finish the next tile's mask before this wait
-        ok = wait_bar(bar(M_READY_A0 + zb), (it >> 1) & 1, abort_flag, kp.status);
-        if (ok) ok = wait_bar(bar(M_READY_B0 + zb), (it >> 1) & 1, abort_flag, kp.status);
-        if (!ok) break;
-        tc_fence_after();
-        // Ydiag = M X_j : K = tokens.  M sits in TMEM as bf16 pairs: the 16 tokens of
-        // K step kk are columns 32 (kk/2) + 8 (kk%2) .. +8 of the Z buffer
-        const uint32_t z_col = tmem + C::COL_Z + zb * 128;
+          const uint32_t w = nyd & 1;
+          const uint64_t dx = sdesc(stage(nyd), kPanel, 1024);
+          const uint32_t z_col = tmem + C::COL_Z + w * 128;
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          tc_mma_ts(tmem + C::COL_YDIAG, z_col + 32 * (kk >> 1) + 8 * (kk & 1),
-                    sdesc(x_base + kk * 2048, kPanel, 1024), ID_YD, kk > 0);
-        tc_commit(bar(YDONE0 + zb));
-        tc_commit(bar(EMPTY0 + s));
-        c = n;
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            tc_mma_ts(z_col + 64, z_col + 8 * kk, dx + ((kk * 2048) >> 4), ID_YD, kk > 0);
+          ++nyd;
+          did = true;
+        } else if (nst < nyd && mbar_test(bar(XW_READY0 + (nst & 1)), (nst >> 1) & 1) &&
+                   mbar_test(bar(PREP0 + (nst & 1)), (nst >> 1) & 1)) {
+          tc_fence_after();
+          const uint32_t w = nst & 1, st = stage(nst);
+          const uint32_t b_base = st + C::X_BYTES, c_base = st + C::X_BYTES + C::BC_BYTES;
+          const uint32_t hb_base = sbase + C::OFF_HB + (C::HB_BUFS == 2 ? w : 0) * C::HB_BYTES;
+          const uint32_t xw_base = sbase + C::OFF_XW + w * kPanel;
+          auto issue_state = [&]() {
+            // H += B_j^T XW : K = tokens; A = the B tile read MN-major (n), B = XW (p)
+            const uint64_t dbm = sdesc(b_base, kPanel, 1024), dxw = sdesc(xw_base, kPanel, 1024);
+#pragma unroll
+            for (int mt = 0; mt < NT; ++mt)
+#pragma unroll
+              for (int kk = 0; kk < kTile / 16; ++kk)
+                tc_mma(tmem + C::COL_H + mt * kPT, dbm + ((2 * mt * kPanel + kk * 2048) >> 4),
+                       dxw + ((kk * 2048) >> 4), ID_ST, 1);
+          };
+          auto issue_yoff = [&]() {
+            // Yoff = C_j Hb : K = state dim; Hb rows are n (K), 128 bytes of p (MN)
+            const uint64_t dc = sdesc(c_base, 16, 1024), dhb = sdesc(hb_base, C::HB_BYTES, 1024);
+#pragma unroll
+            for (int kk = 0; kk < C::NPAD / 16; ++kk)
+              tc_mma(tmem + C::COL_Y + w * kPT, dc + (((kk >> 2) * kPanel + (kk & 3) * 32) >> 4),
+                     dhb + ((kk * 2048) >> 4), ID_YOFF, kk > 0);
+          };
+          if (C::HB_BUFS == 2) {
+            issue_state();
+            tc_commit(bar(STATE_DONE0 + w));
+            issue_yoff();
+            tc_commit(bar(YO_DONE0 + w));
+          } else {
+            // one Hb buffer: the next hand-over may only overwrite it after Yoff read it
+            issue_yoff();
+            issue_state();
+            tc_commit(bar(STATE_DONE0 + w));
+            tc_commit(bar(YO_DONE0 + w));
+          }
+          tc_commit(bar(EMPTY0 + nst % C::NSTAGE));
+          ++nst;
+          did = true;
+        }
+        if (did) {
+          idle = 0;
+          t_last = 0;
+        } else if ((++idle & 15u) != 0) {
+          __nanosleep(32);  // leave issue slots to the epilogue warps of this sub-partition
+        } else {
+          if (*abort_flag) break;
+          const uint64_t now = globaltimer();
+          if (t_last == 0) {
+            t_last = now;
+          } else if (now - t_last > 2000000000ull) {
+            *abort_flag = 1;
+            set_status(kp.status, SSD_ERR_TIMEOUT);
+            break;
+          }
+        }
       }
       // every MMA this thread issued has completed once TEARDOWN fires
       tc_commit(bar(TEARDOWN));
       wait_bar(bar(TEARDOWN), 0, abort_flag, kp.status);
     }
-  } else if (warp < 6) {
-    // ============== epilogue A: decay, state hand-over, mask (blocks 0 and q) ==============
-    const int q = warp & 3;        // TMEM lane quarter of this warp
-    const int r = q * 32 + lane;   // tile row (token) == TMEM lane
+  } else {
+    // ==================== epilogue group w: every other tile, end to end ====================
+    const int w = (warp - 2) >> 2;  // 0: tiles 0, 2, 4, ...  1: tiles 1, 3, 5, ...
+    const int q = warp & 3;         // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;    // tile row (token) == TMEM lane
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t zaddr = tmem + lane_off + C::COL_Z + w * 128;
+    const uint32_t yaddr = tmem + lane_off + C::COL_Y + w * kPT;
+    const uint32_t xw_base = sbase + C::OFF_XW + w * kPanel;  // w o x, then the y staging tile
+    const uint32_t hb_base = sbase + C::OFF_HB + (C::HB_BUFS == 2 ? w : 0) * C::HB_BYTES;
+    float* vw = v_all + 128 * w;
+    float* ws = ws_all + 4 * w;
     const float LOG2E = 1.4426950408889634f;
-    const uint32_t hb0 = sbase + C::OFF_HB;
-
-    auto store_final = [&](int d, int h, int ps, int n, const float* v) {
-      if (!kp.final_states || n >= g.N) return;
-      float* dst = kp.final_states + (((int64_t)d * g.H + h) * g.N + n) * g.P + ps * kPT;
-#pragma unroll
-      for (int c = 0; c < kPT; c += 4)
-        *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+    auto sync_g = [&]() {
+      if (w == 0)
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      else
+        asm volatile("bar.sync 2, 128;" ::: "memory");
     };
-    // documents without tokens: the final state is the initial state
-    for (int u = blockIdx.x; u < kp.units; u += gridDim.x) {
-      const Unit U = unit_of(kp, u);
-      if (U.ntiles != 0 || !kp.final_states) continue;
-      for (int mt = 0; mt < NT; ++mt) {
-        const int n = r + 128 * mt;
-        if (n >= g.N) continue;
-        float v[kPT];
-        const float* src =
-            kp.init ? kp.init + (((int64_t)U.d * g.H + U.h) * g.N + n) * g.P + U.ps * kPT : nullptr;
-#pragma unroll
-        for (int c = 0; c < kPT; ++c) v[c] = src ? src[c] : 0.f;
-        store_final(U.d, U.h, U.ps, n, v);
-      }
-    }
+    if (w == 0) empty_units_final(kp, r, NT);
 
-    // per-tile scalars, loaded one tile ahead
     struct Pre {
       float dt, A, bias, D;
     };
@@ -635,22 +711,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       return p;
     };
 
-    uint32_t it = 0;
     bool ok = true;
-    bool pend = false;
-    int pend_d = 0, pend_h = 0, pend_ps = 0;
     Cursor cur = cursor_first(kp);
+    if (w == 1) cursor_next(kp, cur);
     Cursor nxt = cur;
     cursor_next(kp, nxt);
+    cursor_next(kp, nxt);
     Pre pc = prefetch(cur);
-    for (; cur.valid && ok; ++it) {
-      const Unit& U = cur.U;
+    uint32_t it = w;
+    for (; cur.valid && ok; it += 2) {
+      const Unit U = cur.U;
       const int jt = cur.jt;
       const int len = min(kTile, U.len - jt * kTile);
-      const uint32_t cb = (it & 1) * 128;
-      const Pre pn = prefetch(nxt);  // consumed one tile later
+      const int64_t t0 = U.start + (int64_t)jt * kTile;
+      const uint32_t k = it >> 1, s = it % C::NSTAGE;
+      const Pre pn = prefetch(nxt);  // consumed two tiles later
 
-      // ---- E1: delta and in-tile cumulative log decay (scaled by log2 e) ----
+      // ---- E1: delta and in-tile cumulative log decay (log2 units) ----
       float dl = 0.f, la = 0.f;
       if (r < len) {
         dl = softplus_f(pc.dt + pc.bias);
@@ -662,172 +739,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float t = __shfl_up_sync(0xffffffffu, cs, o);
         if (lane >= o) cs += t;
       }
-      float* ws = wsum + (it & 1) * 4;
       if (lane == 31) ws[q] = cs;
-      // the cs buffer of this parity was last read by epilogue B two tiles ago
-      if (it >= 2) ok = wait_bar(bar(CS_FREE0 + (it & 1)), ((it - 2) >> 1) & 1, abort_flag, kp.status);
-      sync_a();
-      if (!ok) break;
-      for (int w = 0; w < q; ++w) cs += ws[w];
-      const float cs_last = ws[0] + ws[1] + ws[2] + ws[3];
-      const float cs_blockend = __shfl_sync(0xffffffffu, cs, 31);
-      cs_s[cb + r] = cs;
-      dl_s[cb + r] = dl;
-      v_s[cb + r] = ex2(cs_blockend - cs) * dl;
-      w_s[cb + r] = ex2(cs_last - cs) * dl;
-      mbar_arrive(bar(CS_READY0 + (it & 1)));
+      sync_g();
+      const float e0 = ws[0], e1 = e0 + ws[1], e2 = e1 + ws[2], e3 = e2 + ws[3];  // block ends
+      const float base = q == 0 ? 0.f : q == 1 ? e0 : q == 2 ? e1 : e2;
+      const float cs_end = q == 0 ? e0 : q == 1 ? e1 : q == 2 ? e2 : e3;
+      cs += base;
+      vw[r] = ex2(cs_end - cs) * dl;
+      const float wr = ex2(e3 - cs) * dl;  // exp(cs_last - cs) delta
+      const float el = ex2(cs);            // exp(cs)
+      sync_g();
 
-      // ---- E3: state entering the tile -> bf16 copy Hb; decayed copy stays in TMEM ----
-      if (it > 0) ok = wait_bar(bar(STATE_DONE), (it - 1) & 1, abort_flag, kp.status);
-      if (!ok) break;
-      tc_fence_after();
-      {
-        const float decay = ex2(cs_last);
-        const uint32_t hb_base = hb0 + (C::HB_BUFS == 2 ? (it & 1) : 0) * C::HB_BYTES;
-#pragma unroll 1
-        for (int mt = 0; mt < NT; ++mt) {
-          const int n = r + 128 * mt;
-          const uint32_t th = tmem + lane_off + C::COL_H + mt * kPT;
-          float hv[kPT];
-          if (jt == 0) {
-            if (pend) {  // the previous unit's final state is still in TMEM
-              tc_ld32(th, hv);
-              tc_ld32(th + 32, hv + 32);
-              tc_wait_ld();
-              store_final(pend_d, pend_h, pend_ps, n, hv);
-            }
-            const float* src =
-                (kp.init && n < g.N)
-                    ? kp.init + (((int64_t)U.d * g.H + U.h) * g.N + n) * g.P + U.ps * kPT
-                    : nullptr;
-#pragma unroll
-            for (int c = 0; c < kPT; c += 4) {
-              const float4 f = src ? *reinterpret_cast<const float4*>(src + c) : make_float4(0, 0, 0, 0);
-              hv[c] = f.x;
-              hv[c + 1] = f.y;
-              hv[c + 2] = f.z;
-              hv[c + 3] = f.w;
-            }
-          } else {
-            tc_ld32(th, hv);
-            tc_ld32(th + 32, hv + 32);
-            tc_wait_ld();
-          }
-          // Hb row n: the MN-major B operand of Yoff (rows = n, 128 bytes of p)
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_shared_v4(hb_base + swz((uint32_t)n, (uint32_t)c), pack_bf16(hv[8 * c], hv[8 * c + 1]),
-                         pack_bf16(hv[8 * c + 2], hv[8 * c + 3]), pack_bf16(hv[8 * c + 4], hv[8 * c + 5]),
-                         pack_bf16(hv[8 * c + 6], hv[8 * c + 7]));
-#pragma unroll
-          for (int c = 0; c < kPT; ++c) hv[c] *= decay;
-          tc_st32(th, hv);
-          tc_st32(th + 32, hv + 32);
-        }
-        pend = false;
-        tc_wait_st();
-        fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(bar(HB_READY));
-      }
-
-      // ---- E2 (blocks 0 and q; the rest of the causal part is epilogue B's) ----
-      ok = wait_bar(bar(CB_DONE0 + (it & 1)), (it >> 1) & 1, abort_flag, kp.status);
-      if (ok) ok = wait_bar(bar(CS_READY0 + (it & 1)), (it >> 1) & 1, abort_flag, kp.status);
-      if (!ok) break;
-      tc_fence_after();
-      {
-        const uint32_t zaddr = tmem + lane_off + C::COL_Z + (it & 1) * 128;
-        mask_block(zaddr, 0, q, r, cs, cs_s + cb, dl_s + cb, v_s + cb, pc.D);
-        if (q > 0) mask_block(zaddr, q, q, r, cs, cs_s + cb, dl_s + cb, v_s + cb, pc.D);
-#pragma unroll 1
-        for (int cc = q + 1; cc < 4; ++cc) zero_block(zaddr, cc);
-        tc_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(M_READY_A0 + (it & 1)));
-      }
-
-      if (jt == U.ntiles - 1) {
-        pend = true;
-        pend_d = U.d;
-        pend_h = U.h;
-        pend_ps = U.ps;
-      }
-      cur = nxt;
-      cursor_next(kp, nxt);
-      pc = pn;
-    }
-    if (ok && pend) {
-      ok = wait_bar(bar(STATE_DONE), (it - 1) & 1, abort_flag, kp.status);
-      if (ok) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int mt = 0; mt < NT; ++mt) {
-          float hv[kPT];
-          const uint32_t th = tmem + lane_off + C::COL_H + mt * kPT;
-          tc_ld32(th, hv);
-          tc_ld32(th + 32, hv + 32);
-          tc_wait_ld();
-          store_final(pend_d, pend_h, pend_ps, r + 128 * mt, hv);
-        }
-      }
-    }
-  } else {
-    // ========= epilogue B: weighted input, mask blocks 1..q-1, outputs =========
-    const int q = warp & 3;
-    const int r = q * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const uint32_t xw_base = sbase + C::OFF_XW;
-    uint32_t it = 0;
-    bool ok = true;
-    bool prev = false;
-    int64_t prev_t0 = 0;
-    int prev_len = 0, prev_h = 0, prev_ps = 0;
-    float prev_el = 0.f;
-
-    // output of tile pit: y = exp(cs) Yoff + Ydiag
-    auto emit = [&](uint32_t pit) -> bool {
-      if (!wait_bar(bar(YDONE0 + (pit & 1)), (pit >> 1) & 1, abort_flag, kp.status)) return false;
-      tc_fence_after();
-      const bool valid = r < prev_len;
-      __nv_bfloat16* dst = kp.y + ((prev_t0 + r) * g.H + prev_h) * (int64_t)g.P + prev_ps * kPT;
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        float yo[32], yd[32];
-        tc_ld32(tmem + lane_off + C::COL_YOFF + half * 32, yo);
-        tc_ld32(tmem + lane_off + C::COL_YDIAG + half * 32, yd);
-        tc_wait_ld();
-        if (valid) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint4 v;
-            v.x = pack_bf16(fmaf(prev_el, yo[c + 0], yd[c + 0]), fmaf(prev_el, yo[c + 1], yd[c + 1]));
-            v.y = pack_bf16(fmaf(prev_el, yo[c + 2], yd[c + 2]), fmaf(prev_el, yo[c + 3], yd[c + 3]));
-            v.z = pack_bf16(fmaf(prev_el, yo[c + 4], yd[c + 4]), fmaf(prev_el, yo[c + 5], yd[c + 5]));
-            v.w = pack_bf16(fmaf(prev_el, yo[c + 6], yd[c + 6]), fmaf(prev_el, yo[c + 7], yd[c + 7]));
-            *reinterpret_cast<uint4*>(dst + half * 32 + c) = v;
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(Y_FREE));
-      return true;
-    };
-
-    for (Cursor c = cursor_first(kp); c.valid && ok; cursor_next(kp, c), ++it) {
-      const uint32_t s = it % C::NSTAGE, k = it / C::NSTAGE, cb = (it & 1) * 128;
-      // the four warps of this group finish a tile (and all its barrier arrivals)
-      // before any of them starts the next, so arrivals never mix tiles
-      sync_b();
-      // ---- E4: XW = w o x_j ----
-      ok = wait_bar(bar(CS_READY0 + (it & 1)), (it >> 1) & 1, abort_flag, kp.status);
-      if (!ok) break;
-      const float wr = w_s[cb + r];
-      const float cs_r = cs_s[cb + r];
-      const float el = ex2(cs_r);
-      ok = wait_bar(bar(FULL0 + s), k & 1, abort_flag, kp.status);
-      // XW is free once the previous tile's state update has read it
-      if (ok && it > 0) ok = wait_bar(bar(STATE_DONE), (it - 1) & 1, abort_flag, kp.status);
+      // ---- E4: XW = w o x_j (MN-major B operand of the state update) ----
+      ok = wait_bar(bar(FULL0 + s), (it / C::NSTAGE) & 1, abort_flag, kp.status);
       if (!ok) break;
       {
         const uint32_t xrow = sbase + s * C::STAGE_BYTES;
@@ -843,42 +767,125 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_async_smem();
-      mbar_arrive(bar(XW_READY));
+      mbar_arrive(bar(XW_READY0 + w));
 
-      // ---- E2 (off-diagonal blocks 1..q-1 of this lane quarter) ----
-      ok = wait_bar(bar(CB_DONE0 + (it & 1)), (it >> 1) & 1, abort_flag, kp.status);
+      // ---- E2: decay mask of the diagonal block, over C B^T in TMEM ----
+      ok = wait_bar(bar(CB_DONE0 + w), k & 1, abort_flag, kp.status);
       if (!ok) break;
       tc_fence_after();
-      {
-        const uint32_t zaddr = tmem + lane_off + C::COL_Z + (it & 1) * 128;
+      if (q > 0) mask_off(zaddr, 0, cs, e0, vw);
+      if (q > 1) mask_off(zaddr, 1, cs, e1, vw);
+      if (q > 2) mask_off(zaddr, 2, cs, e2, vw);
+      mask_diag(zaddr, q, lane, cs, dl, pc.D);
 #pragma unroll 1
-        for (int cc = 1; cc < q; ++cc)
-          mask_block(zaddr, cc, q, r, cs_r, cs_s + cb, dl_s + cb, v_s + cb, 0.f);
-        tc_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(M_READY_B0 + (it & 1)));
-      }
-      mbar_arrive(bar(CS_FREE0 + (it & 1)));  // done with this tile's cs buffer
+      for (int cc = q + 1; cc < 4; ++cc) zero_block(zaddr, cc);
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(M_READY0 + w));
 
-      // ---- E5 of the previous tile ----
-      if (prev && !emit(it - 1)) {
-        ok = false;
-        break;
+      // ---- E3: the state entering the tile (after the previous tile's update) ----
+      if (it > 0) {
+        const int pb = (C::HB_BUFS == 2 ? STATE_DONE0 : YO_DONE0) + (w ^ 1);
+        ok = wait_bar(bar(pb), ((it - 1) >> 1) & 1, abort_flag, kp.status);
+        if (!ok) break;
       }
-      prev = true;
-      prev_t0 = c.U.start + (int64_t)c.jt * kTile;
-      prev_len = min(kTile, c.U.len - c.jt * kTile);
-      prev_h = c.U.h;
-      prev_ps = c.U.ps;
-      prev_el = el;
+      tc_fence_after();
+      {
+        const float decay = ex2(e3);
+        int pu = -1;
+        if (jt == 0 && it > 0) pu = prev_unit_with_tiles(kp, cur.u);
+        const Unit P = pu >= 0 ? unit_of(kp, pu) : U;
+#pragma unroll 1
+        for (int mt = 0; mt < NT; ++mt) {
+          const int n = r + 128 * mt;
+          const uint32_t th = tmem + lane_off + C::COL_H + mt * kPT;
+          if (jt == 0) {
+            // the previous unit's final state is still in TMEM
+            if (pu >= 0) tmem_state_to_final(kp, th, P.d, P.h, P.ps, n);
+            enter_unit_row(kp, th, hb_base, U.d, U.h, U.ps, n, decay);
+            continue;
+          }
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            float hv[32];
+            tc_ld32(th + 32 * half, hv);
+            tc_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              st_shared_v4(hb_base + swz((uint32_t)n, (uint32_t)(4 * half + c)),
+                           pack_bf16(hv[8 * c], hv[8 * c + 1]), pack_bf16(hv[8 * c + 2], hv[8 * c + 3]),
+                           pack_bf16(hv[8 * c + 4], hv[8 * c + 5]), pack_bf16(hv[8 * c + 6], hv[8 * c + 7]));
+#pragma unroll
+            for (int c = 0; c < 32; ++c) hv[c] *= decay;
+            tc_st32(th + 32 * half, hv);
+          }
+        }
+      }
+      tc_wait_st();
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(PREP0 + w));
+
+      // ---- E5: y = exp(cs) Yoff + Ydiag, staged in smem, coalesced stores ----
+      ok = wait_bar(bar(YO_DONE0 + w), k & 1, abort_flag, kp.status);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        float yo[32], yd[32];
+        tc_ld32(yaddr + 32 * half, yo);
+        tc_ld32(zaddr + 64 + 32 * half, yd);
+        tc_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(xw_base + swz((uint32_t)r, (uint32_t)(4 * half + c)),
+                       pack_bf16(fmaf(el, yo[8 * c + 0], yd[8 * c + 0]), fmaf(el, yo[8 * c + 1], yd[8 * c + 1])),
+                       pack_bf16(fmaf(el, yo[8 * c + 2], yd[8 * c + 2]), fmaf(el, yo[8 * c + 3], yd[8 * c + 3])),
+                       pack_bf16(fmaf(el, yo[8 * c + 4], yd[8 * c + 4]), fmaf(el, yo[8 * c + 5], yd[8 * c + 5])),
+                       pack_bf16(fmaf(el, yo[8 * c + 6], yd[8 * c + 6]), fmaf(el, yo[8 * c + 7], yd[8 * c + 7])));
+      }
+      tc_fence_before();
+      mbar_arrive(bar(Z_FREE0 + w));  // Z (mask + Ydiag) and Yoff are read: next C B^T may land
+      sync_g();
+      {
+        // 16-byte chunk e of the 128 x 128-byte tile: row e/8, chunk e%8; a warp
+        // instruction covers four whole rows
+        const int tid = q * 32 + lane;
+        __nv_bfloat16* ybase = kp.y + (int64_t)U.h * g.P + U.ps * kPT;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = tid + 128 * i, row = e >> 3, c = e & 7;
+          if (row < len) {
+            const uint4 v = ld_shared_v4(xw_base + swz((uint32_t)row, (uint32_t)c));
+            *reinterpret_cast<uint4*>(ybase + (t0 + row) * (int64_t)g.H * g.P + c * 8) = v;
+          }
+        }
+      }
+
+      cur = nxt;
+      cursor_next(kp, nxt);
+      cursor_next(kp, nxt);
+      pc = pn;
     }
-    if (ok && prev) emit(it - 1);
+    // the group that would own the next tile hands out the last unit's final state
+    if (ok && ntiles > 0 && (ntiles & 1u) == (uint32_t)w && last_unit >= 0) {
+      const uint32_t lt = ntiles - 1;
+      const int pb = (C::HB_BUFS == 2 ? STATE_DONE0 : YO_DONE0) + (w ^ 1);
+      ok = wait_bar(bar(pb), (lt >> 1) & 1, abort_flag, kp.status);
+      if (ok) {
+        tc_fence_after();
+        const Unit L = unit_of(kp, last_unit);
+#pragma unroll 1
+        for (int mt = 0; mt < NT; ++mt)
+          tmem_state_to_final(kp, tmem + lane_off + C::COL_H + mt * kPT, L.d, L.h, L.ps, r + 128 * mt);
+      }
+    }
   }
 
   // ---- teardown ----
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
