@@ -144,37 +144,26 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- ranks
 def dist_setup(n):
+    """One process per GPU; the process group only coordinates (barrier, max time)."""
     import torch
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from structured_state_space_chunked_b200 import dist as sdist
+    rank, world, local = sdist.env_ranks()
     if world != n:
         raise SystemExit(f"--gpus {n} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-        pg = dist
+    pg = sdist.init("nccl", timeout_s=120, device=torch.device("cuda", local))
     return rank, world, local, pg
 
 
 def barrier(pg):
-    import torch
-    if pg is not None:
-        pg.barrier()
-    torch.cuda.synchronize()
+    from structured_state_space_chunked_b200 import dist as sdist
+    sdist.barrier(pg)
 
 
 def max_over_ranks(pg, v):
     import torch
-    if pg is None:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    return float(t.item())
+    from structured_state_space_chunked_b200 import dist as sdist
+    return sdist.max_over_ranks(v, pg, device=torch.device("cuda", torch.cuda.current_device()))
 
 
 # ----------------------------------------------------------------------------- oracle arm

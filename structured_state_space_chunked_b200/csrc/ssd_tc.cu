@@ -301,27 +301,30 @@ struct Cursor {
   bool valid;
   Unit U;
 };
-__device__ __noinline__ void cursor_next(const KParams& kp, Cursor& c) {
-  if (c.valid && c.jt + 1 < c.U.ntiles) {
+// The next unit with tokens after unit u in this CTA's stream (u < 0: none).
+__device__ __noinline__ int next_unit_with_tiles(const KParams& kp, int u) {
+  for (u += gridDim.x; u < kp.units; u += gridDim.x)
+    if (unit_of(kp, u).ntiles > 0) return u;
+  return -1;
+}
+// Advance to the next tile: within a unit only the tile index moves.
+__device__ __forceinline__ void cursor_next(const KParams& kp, Cursor& c) {
+  if (!c.valid) return;
+  if (c.jt + 1 < c.U.ntiles) {
     ++c.jt;
     return;
   }
-  for (c.u += gridDim.x; c.u < kp.units; c.u += gridDim.x) {
-    c.U = unit_of(kp, c.u);
-    if (c.U.ntiles > 0) {
-      c.jt = 0;
-      c.valid = true;
-      return;
-    }
-  }
-  c.valid = false;
+  c.u = next_unit_with_tiles(kp, c.u);
+  c.valid = c.u >= 0;
+  c.jt = 0;
+  if (c.valid) c.U = unit_of(kp, c.u);
 }
 __device__ __forceinline__ Cursor cursor_first(const KParams& kp) {
   Cursor c;
-  c.u = (int)blockIdx.x - (int)gridDim.x;
+  c.u = next_unit_with_tiles(kp, (int)blockIdx.x - (int)gridDim.x);
   c.jt = 0;
-  c.valid = false;
-  cursor_next(kp, c);
+  c.valid = c.u >= 0;
+  if (c.valid) c.U = unit_of(kp, c.u);
   return c;
 }
 
@@ -482,7 +485,7 @@ __device__ __noinline__ int prev_unit_with_tiles(const KParams& kp, int u) {
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_tc_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                 const __grid_constant__ CUtensorMap tm_c, const KParams kp) {
+                 const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ KParams kp) {
   using C = Cfg<NT>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = su32(smem);
@@ -717,23 +720,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     Cursor nxt = cur;
     cursor_next(kp, nxt);
     cursor_next(kp, nxt);
-    Pre pc = prefetch(cur);
-    uint32_t it = w;
-    for (; cur.valid && ok; it += 2) {
-      const Unit U = cur.U;
-      const int jt = cur.jt;
-      const int len = min(kTile, U.len - jt * kTile);
-      const int64_t t0 = U.start + (int64_t)jt * kTile;
-      const uint32_t k = it >> 1, s = it % C::NSTAGE;
-      const Pre pn = prefetch(nxt);  // consumed two tiles later
 
-      // ---- E1: delta and in-tile cumulative log decay (log2 units) ----
-      float dl = 0.f, la = 0.f;
+    // E1 of a tile: delta, in-tile cumulative log decay (log2 units), the per-column
+    // factor v (shared through smem), the input weight w and exp(cs) for the output.
+    float cs = 0.f, dl = 0.f, wr = 0.f, el = 0.f, e0 = 0.f, e1 = 0.f, e2 = 0.f, e3 = 0.f, Dh = 0.f;
+    auto stage1 = [&](const Cursor& c, const Pre& p) {
+      const int len = min(kTile, c.U.len - c.jt * kTile);
+      float la = 0.f;
+      dl = 0.f;
       if (r < len) {
-        dl = softplus_f(pc.dt + pc.bias);
-        la = dl * pc.A * LOG2E;
+        dl = softplus_f(p.dt + p.bias);
+        la = dl * p.A * LOG2E;
       }
-      float cs = la;
+      cs = la;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float t = __shfl_up_sync(0xffffffffu, cs, o);
@@ -741,18 +740,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (lane == 31) ws[q] = cs;
       sync_g();
-      const float e0 = ws[0], e1 = e0 + ws[1], e2 = e1 + ws[2], e3 = e2 + ws[3];  // block ends
+      e0 = ws[0];
+      e1 = e0 + ws[1];
+      e2 = e1 + ws[2];
+      e3 = e2 + ws[3];  // block ends; e3 = cs of the tile's last row
       const float base = q == 0 ? 0.f : q == 1 ? e0 : q == 2 ? e1 : e2;
       const float cs_end = q == 0 ? e0 : q == 1 ? e1 : q == 2 ? e2 : e3;
       cs += base;
       vw[r] = ex2(cs_end - cs) * dl;
-      const float wr = ex2(e3 - cs) * dl;  // exp(cs_last - cs) delta
-      const float el = ex2(cs);            // exp(cs)
+      wr = ex2(e3 - cs) * dl;  // exp(cs_last - cs) delta
+      el = ex2(cs);            // exp(cs)
+      Dh = p.D;
       sync_g();
+    };
 
-      // ---- E4: XW = w o x_j (MN-major B operand of the state update) ----
+    uint32_t it = w;
+    if (cur.valid) stage1(cur, prefetch(cur));
+    for (; cur.valid && ok; it += 2) {
+      const Unit U = cur.U;
+      const int jt = cur.jt;
+      const int len = min(kTile, U.len - jt * kTile);
+      const int64_t t0 = U.start + (int64_t)jt * kTile;
+      const uint32_t k = it >> 1, s = it % C::NSTAGE;
+      const Pre pn = prefetch(nxt);  // consumed by E1 of the next tile, later in this iteration
+
+      // With two stages, stage it % 2 == w only ever holds this group's tiles, so the
+      // FULL parity test is unambiguous right away.  With one stage the group sees
+      // every other fill: it first waits for this tile's C B^T, which implies the
+      // load landed and that the stage cannot be refilled before this tile's state
+      // update, so the parity test is then unambiguous too.
+      if (C::NSTAGE == 1) {
+        ok = wait_bar(bar(CB_DONE0 + w), k & 1, abort_flag, kp.status);
+        if (!ok) break;
+      }
       ok = wait_bar(bar(FULL0 + s), (it / C::NSTAGE) & 1, abort_flag, kp.status);
       if (!ok) break;
+
+      // ---- E4: XW = w o x_j (MN-major B operand of the state update) ----
       {
         const uint32_t xrow = sbase + s * C::STAGE_BYTES;
 #pragma unroll
@@ -770,13 +794,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(XW_READY0 + w));
 
       // ---- E2: decay mask of the diagonal block, over C B^T in TMEM ----
-      ok = wait_bar(bar(CB_DONE0 + w), k & 1, abort_flag, kp.status);
-      if (!ok) break;
+      if (C::NSTAGE != 1) {
+        ok = wait_bar(bar(CB_DONE0 + w), k & 1, abort_flag, kp.status);
+        if (!ok) break;
+      }
       tc_fence_after();
       if (q > 0) mask_off(zaddr, 0, cs, e0, vw);
       if (q > 1) mask_off(zaddr, 1, cs, e1, vw);
       if (q > 2) mask_off(zaddr, 2, cs, e2, vw);
-      mask_diag(zaddr, q, lane, cs, dl, pc.D);
+      mask_diag(zaddr, q, lane, cs, dl, Dh);
 #pragma unroll 1
       for (int cc = q + 1; cc < 4; ++cc) zero_block(zaddr, cc);
       tc_wait_st();
@@ -826,6 +852,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(PREP0 + w));
 
+      // ---- E1 of this group's next tile, while the tensor cores finish this one ----
+      const float el_cur = el;
+      if (nxt.valid) stage1(nxt, pn);
+
       // ---- E5: y = exp(cs) Yoff + Ydiag, staged in smem, coalesced stores ----
       ok = wait_bar(bar(YO_DONE0 + w), k & 1, abort_flag, kp.status);
       if (!ok) break;
@@ -839,10 +869,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           st_shared_v4(xw_base + swz((uint32_t)r, (uint32_t)(4 * half + c)),
-                       pack_bf16(fmaf(el, yo[8 * c + 0], yd[8 * c + 0]), fmaf(el, yo[8 * c + 1], yd[8 * c + 1])),
-                       pack_bf16(fmaf(el, yo[8 * c + 2], yd[8 * c + 2]), fmaf(el, yo[8 * c + 3], yd[8 * c + 3])),
-                       pack_bf16(fmaf(el, yo[8 * c + 4], yd[8 * c + 4]), fmaf(el, yo[8 * c + 5], yd[8 * c + 5])),
-                       pack_bf16(fmaf(el, yo[8 * c + 6], yd[8 * c + 6]), fmaf(el, yo[8 * c + 7], yd[8 * c + 7])));
+                       pack_bf16(fmaf(el_cur, yo[8 * c + 0], yd[8 * c + 0]), fmaf(el_cur, yo[8 * c + 1], yd[8 * c + 1])),
+                       pack_bf16(fmaf(el_cur, yo[8 * c + 2], yd[8 * c + 2]), fmaf(el_cur, yo[8 * c + 3], yd[8 * c + 3])),
+                       pack_bf16(fmaf(el_cur, yo[8 * c + 4], yd[8 * c + 4]), fmaf(el_cur, yo[8 * c + 5], yd[8 * c + 5])),
+                       pack_bf16(fmaf(el_cur, yo[8 * c + 6], yd[8 * c + 6]), fmaf(el_cur, yo[8 * c + 7], yd[8 * c + 7])));
       }
       tc_fence_before();
       mbar_arrive(bar(Z_FREE0 + w));  // Z (mask + Ydiag) and Yoff are read: next C B^T may land
@@ -861,11 +891,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      sync_g();  // the staging tile is read before the next tile's w o x lands there
 
       cur = nxt;
       cursor_next(kp, nxt);
       cursor_next(kp, nxt);
-      pc = pn;
     }
     // the group that would own the next tile hands out the last unit's final state
     if (ok && ntiles > 0 && (ntiles & 1u) == (uint32_t)w && last_unit >= 0) {

@@ -1,0 +1,81 @@
+"""Multi-process plumbing for running the SSD forward on several GPUs.
+
+The forward pass partitions cleanly: documents (batch rows, or packed documents)
+and heads are independent, so ranks need no data-path collective.  A global
+batch is split into contiguous document ranges, one per rank, and every rank
+runs ``ssd_forward`` on its range with its own handle.  The only collectives
+are for coordination: a barrier around timed regions and a max over ranks of
+the measured time.  One process per GPU; rank/world come from the usual
+``RANK``/``WORLD_SIZE``/``LOCAL_RANK`` environment of ``torchrun``.
+"""
+
+from __future__ import annotations
+
+import datetime
+import os
+from typing import Optional, Tuple
+
+import torch
+import torch.distributed as dist
+
+
+def env_ranks() -> Tuple[int, int, int]:
+    """(rank, world_size, local_rank) from the launcher's environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init(backend: str = "nccl", timeout_s: float = 120.0, device: Optional[torch.device] = None):
+    """Join the process group when WORLD_SIZE > 1; returns the group module or None."""
+    rank, world, _ = env_ranks()
+    if world <= 1:
+        return None
+    kw = {}
+    if backend == "nccl" and device is not None:
+        kw["device_id"] = device
+    dist.init_process_group(backend, rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    return dist
+
+
+def shard_range(n: int, world: int, rank: int) -> Tuple[int, int]:
+    """Contiguous [start, stop) share of n independent items for `rank` of `world`.
+
+    Shares differ by at most one item and cover 0..n-1 exactly once.
+    """
+    if world <= 0 or not (0 <= rank < world):
+        raise ValueError("bad rank/world")
+    base, extra = divmod(n, world)
+    start = rank * base + min(rank, extra)
+    return start, start + base + (1 if rank < extra else 0)
+
+
+def shard_documents(cu_seqlens, world: int, rank: int):
+    """This rank's documents of a packed row: (token_start, token_stop, local cu_seqlens).
+
+    Documents are split into contiguous ranges balanced by document count; the
+    local cu_seqlens is rebased to start at 0.
+    """
+    import numpy as np
+
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    d0, d1 = shard_range(len(cu) - 1, world, rank)
+    t0, t1 = int(cu[d0]), int(cu[d1])
+    return t0, t1, (cu[d0:d1 + 1] - t0).astype(np.int32)
+
+
+def barrier(group=None, device_sync: bool = True) -> None:
+    if group is not None:
+        group.barrier()
+    if device_sync and torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def max_over_ranks(value: float, group=None, device: Optional[torch.device] = None) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity without a group)."""
+    if group is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    group.all_reduce(t, op=group.ReduceOp.MAX)
+    return float(t.item())
