@@ -589,35 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t idle = 0;
       while (nst < ntiles) {
         bool did = false;
-        if (ncb < ntiles && ncb < nyd + 2 &&
-            mbar_test(bar(FULL0 + ncb % C::NSTAGE), (ncb / C::NSTAGE) & 1) &&
-            (ncb < 2 || mbar_test(bar(Z_FREE0 + (ncb & 1)), ((ncb - 2) >> 1) & 1))) {
-          // Z[w] = C_j B_j^T : K = state dim
-          tc_fence_after();
-          const uint32_t st = stage(ncb), w = ncb & 1;
-          const uint64_t dc = sdesc(st + C::X_BYTES + C::BC_BYTES, 16, 1024);
-          const uint64_t db = sdesc(st + C::X_BYTES, 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < C::NPAD / 16; ++kk) {
-            const uint64_t off = ((kk >> 2) * kPanel + (kk & 3) * 32) >> 4;
-            tc_mma(tmem + C::COL_Z + w * 128, dc + off, db + off, ID_CB, kk > 0);
-          }
-          tc_commit(bar(CB_DONE0 + w));
-          ++ncb;
-          did = true;
-        } else if (nyd < ncb && mbar_test(bar(M_READY0 + (nyd & 1)), (nyd >> 1) & 1)) {
-          // Ydiag = M X_j : K = tokens.  M sits in TMEM as bf16 pairs (the 16 tokens of
-          // K step kk in columns 8kk..8kk+7 of the Z buffer); Ydiag goes next to it
-          tc_fence_after();
-          const uint32_t w = nyd & 1;
-          const uint64_t dx = sdesc(stage(nyd), kPanel, 1024);
-          const uint32_t z_col = tmem + C::COL_Z + w * 128;
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            tc_mma_ts(z_col + 64, z_col + 8 * kk, dx + ((kk * 2048) >> 4), ID_YD, kk > 0);
-          ++nyd;
-          did = true;
-        } else if (nst < nyd && mbar_test(bar(XW_READY0 + (nst & 1)), (nst >> 1) & 1) &&
+        // the state update is on the chain between the two epilogue groups: serve it first
+        if (nst < nyd && mbar_test(bar(XW_READY0 + (nst & 1)), (nst >> 1) & 1) &&
                    mbar_test(bar(PREP0 + (nst & 1)), (nst >> 1) & 1)) {
           tc_fence_after();
           const uint32_t w = nst & 1, st = stage(nst);
@@ -656,6 +629,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(bar(EMPTY0 + nst % C::NSTAGE));
           ++nst;
+          did = true;
+        } else if (ncb < ntiles && ncb < nyd + 2 &&
+            mbar_test(bar(FULL0 + ncb % C::NSTAGE), (ncb / C::NSTAGE) & 1) &&
+            (ncb < 2 || mbar_test(bar(Z_FREE0 + (ncb & 1)), ((ncb - 2) >> 1) & 1))) {
+          // Z[w] = C_j B_j^T : K = state dim
+          tc_fence_after();
+          const uint32_t st = stage(ncb), w = ncb & 1;
+          const uint64_t dc = sdesc(st + C::X_BYTES + C::BC_BYTES, 16, 1024);
+          const uint64_t db = sdesc(st + C::X_BYTES, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < C::NPAD / 16; ++kk) {
+            const uint64_t off = ((kk >> 2) * kPanel + (kk & 3) * 32) >> 4;
+            tc_mma(tmem + C::COL_Z + w * 128, dc + off, db + off, ID_CB, kk > 0);
+          }
+          tc_commit(bar(CB_DONE0 + w));
+          ++ncb;
+          did = true;
+        } else if (nyd < ncb && mbar_test(bar(M_READY0 + (nyd & 1)), (nyd >> 1) & 1)) {
+          // Ydiag = M X_j : K = tokens.  M sits in TMEM as bf16 pairs (the 16 tokens of
+          // K step kk in columns 8kk..8kk+7 of the Z buffer); Ydiag goes next to it
+          tc_fence_after();
+          const uint32_t w = nyd & 1;
+          const uint64_t dx = sdesc(stage(nyd), kPanel, 1024);
+          const uint32_t z_col = tmem + C::COL_Z + w * 128;
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            tc_mma_ts(z_col + 64, z_col + 8 * kk, dx + ((kk * 2048) >> 4), ID_YD, kk > 0);
+          ++nyd;
           did = true;
         }
         if (did) {
