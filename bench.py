@@ -61,7 +61,7 @@ def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "structured_state_space_chunked_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".h")):
+        if fn.endswith((".cu", ".cuh", ".h")):
             with open(os.path.join(csrc, fn), "rb") as f:
                 h.update(f.read())
     return h.hexdigest()[:16]

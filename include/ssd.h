@@ -78,7 +78,14 @@ enum {
 
 /* handle options (ssd_set_option) */
 enum {
-  SSD_OPT_FORCE_PATH = 1 /* value: SSD_PATH_AUTO (default), SSD_PATH_SIMT or SSD_PATH_TC */
+  SSD_OPT_FORCE_PATH = 1, /* value: SSD_PATH_AUTO (default), SSD_PATH_SIMT or SSD_PATH_TC */
+  /* value: 64 (default) or 128, the column width of the tensor-core kernel's work
+   * units.  128-column units pair two heads of P = 64 that share a B/C group (or
+   * take 128 columns of one head with P = 128 or 256), computing C B^T once for
+   * the pair and the state update and left factors as N = 128 products; they need
+   * dstate <= 128.  On a shape they do not cover, ssd_forward returns
+   * SSD_ERR_UNSUPPORTED.  Both widths compute the same result. */
+  SSD_OPT_TC_UNIT_COLUMNS = 2
 };
 
 /*

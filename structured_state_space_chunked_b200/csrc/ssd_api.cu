@@ -15,6 +15,7 @@ struct ssd_handle_s {
   int device;
   int num_sms;
   int force_path;
+  int tc_unit_columns;  // 64 or 128
   int* status;          // device status word (first error code, 0 = ok)
   void* ws;             // stream-ordered workspace
   size_t ws_bytes;
@@ -131,6 +132,7 @@ int ssd_create(const ssd_desc_t* desc, ssd_handle_t* out) {
   h->device = dev;
   h->num_sms = sms;
   h->force_path = SSD_PATH_AUTO;
+  h->tc_unit_columns = 64;
   cudaError_t e = cudaMalloc(&h->status, sizeof(int) * 4);
   if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int) * 4);
   if (e != cudaSuccess) {
@@ -148,6 +150,11 @@ int ssd_set_option(ssd_handle_t h, int option, int value) {
     if (value != SSD_PATH_AUTO && value != SSD_PATH_SIMT && value != SSD_PATH_TC)
       return SSD_ERR_INVALID_ARG;
     h->force_path = value;
+    return SSD_OK;
+  }
+  if (option == SSD_OPT_TC_UNIT_COLUMNS) {
+    if (value != 64 && value != 128) return SSD_ERR_INVALID_ARG;
+    h->tc_unit_columns = value;
     return SSD_OK;
   }
   return SSD_ERR_INVALID_ARG;
@@ -174,6 +181,8 @@ int ssd_forward(ssd_handle_t h, const void* x, const void* dt, const float* A, c
   make_geom(d, chunk_size, cu_seqlens != nullptr, num_docs, &g);
   const int path = choose_path(d, g, h->force_path);
   if (path < 0) return path;
+  if (path == SSD_PATH_TC && h->tc_unit_columns == 128 && !ssd::tc_wide_supported(g))
+    return SSD_ERR_UNSUPPORTED;
 
   int cur = 0;
   if (cudaGetDevice(&cur) != cudaSuccess) return SSD_ERR_CUDA;
@@ -195,7 +204,7 @@ int ssd_forward(ssd_handle_t h, const void* x, const void* dt, const float* A, c
   ssd::Args a{x, dt, A, B, C, D, dt_bias, initial_states, cu_seqlens, y, final_states};
   cudaError_t e;
   if (path == SSD_PATH_TC) {
-    e = ssd::tc_forward(g, a, h->ws, h->status, stream, h->num_sms);
+    e = ssd::tc_forward(g, a, h->ws, h->status, stream, h->num_sms, h->tc_unit_columns);
   } else {
     ssd::SimtWorkspace ws;
     ssd::simt_carve_workspace(g, h->ws, &ws);

@@ -80,6 +80,11 @@ int tc_units(const Geom& g);
 int tc_kernels(const Geom& g);
 size_t tc_workspace_bytes(const Geom& g);
 cudaError_t tc_forward(const Geom& g, const Args& a, void* workspace, int* status,
-                       cudaStream_t stream, int num_sms);
+                       cudaStream_t stream, int num_sms, int unit_columns);
+// 128-column units (ssd_tc_wide.cu): tc_forward with unit_columns == 128
+bool tc_wide_supported(const Geom& g);
+int tc_wide_units(const Geom& g);
+cudaError_t tc_wide_forward(const Geom& g, const Args& a, int* status, cudaStream_t stream,
+                            int num_sms);
 
 }  // namespace ssd

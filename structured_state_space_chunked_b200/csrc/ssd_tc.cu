@@ -27,26 +27,28 @@
 // a strictly lower block is rank one, §3.2.2), which equals the quadratic form
 // up to rounding.
 //
-// Roles: warp 0 issues TMA loads (x/B/C tiles, double-buffered when they fit),
-// warp 1 owns TMEM and one thread issues every tcgen05.mma, warps 2..5
-// (epilogue A) compute the cumulative decay, hand the state over and build the
-// decay-masked operand M in TMEM (over C B^T, as bf16), warps 6..9 (epilogue B)
-// build the weighted input w o x and write the outputs.  The two epilogue groups
-// work on consecutive tiles at once.  Every mbarrier wait is bounded: on expiry
-// the CTA records SSD_ERR_TIMEOUT in the status word and unwinds.
+// Roles: warp 0 owns TMEM and one of its threads issues every tcgen05.mma, warp 1
+// issues the TMA loads (x/B/C tiles, double-buffered when they fit), and two
+// epilogue groups of four warps (2..5 and 6..9) take alternate tiles end to end:
+// cumulative decay, w o x, the decay-masked operand M (written over C B^T in
+// TMEM, as bf16), the state hand-over and the outputs.  This kernel takes 64-wide
+// column units; ssd_tc_wide.cu takes 128-wide ones where the shape allows.  Every
+// mbarrier wait is bounded: on expiry the CTA records SSD_ERR_TIMEOUT in the status
+// word and unwinds.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "ssd_internal.h"
+#include "tc_common.cuh"
 
 namespace ssd {
 namespace {
+using namespace tc;
 
 constexpr int kTile = 128;          // tokens per tile
 constexpr int kPT = 64;             // head-dim columns per unit
 constexpr int kThreads = 320;       // 10 warps: MMA, TMA, two epilogue groups of 4
-constexpr uint32_t kPanel = 16384;  // one 128-row x 128-byte SW128 panel
 
 template <int NT>
 struct Cfg {
@@ -89,172 +91,6 @@ enum Bar {
   YO_DONE0, YO_DONE1,       // Ydiag and Yoff done (MMA -> group; other group if one Hb)
   TEARDOWN, NBAR
 };
-
-// ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ uint32_t su32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t a) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(a), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-// D(tmem) (+)= A(smem desc) * B(smem desc)
-__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                       uint32_t accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum)
-      : "memory");
-}
-// D(tmem) (+)= A(tmem) * B(smem desc)
-__device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                          uint32_t accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum)
-      : "memory");
-}
-__device__ __forceinline__ void tc_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tc_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-// 32 consecutive TMEM columns of this warp's 32 lanes -> 32 registers per thread
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, float* v) {
-  uint32_t* r = reinterpret_cast<uint32_t*>(v);
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tc_st32(uint32_t taddr, const float* v) {
-  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
-                                       int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
-                                       int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-// named barriers of epilogue group A (warps 2..5) and group B (warps 6..9)
-__device__ __forceinline__ void sync_a() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-__device__ __forceinline__ void sync_b() {
-  asm volatile("bar.sync 2, 128;" ::: "memory");
-}
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z,
-                                             uint32_t w) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z),
-               "r"(w)
-               : "memory");
-}
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(a));
-  return v;
-}
-
-// byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128B-swizzled panel
-__device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c) {
-  return r * 128u + ((c ^ (r & 7u)) << 4);
-}
-
-// tcgen05 shared-memory matrix descriptor, 128-byte swizzle (sm100 layout type 2)
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// instruction descriptor: bf16 x bf16 -> f32, M x N, operand majorness (1 = MN-major)
-__host__ __device__ constexpr uint32_t idesc(int M, int N, int a_mn, int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
 
 struct KParams {
   Geom g;
@@ -453,16 +289,6 @@ __device__ __forceinline__ void zero_block(uint32_t zaddr, int cc) {
   tc_st16(zaddr + 16 * cc, pk);
 }
 
-__device__ __forceinline__ bool mbar_test(uint32_t a, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(a), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
 
 // Number of tiles this CTA processes, and the last unit of its stream with tokens.
 __device__ __noinline__ uint32_t count_tiles(const KParams& kp, int* last_unit) {
@@ -702,13 +528,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (w == 0) empty_units_final(kp, r, NT);
 
     struct Pre {
-      float dt, A, bias, D;
+      uint32_t dt;  // raw bf16 bits: converted only in E1, so the load latency stays hidden
+      float A, bias, D;
     };
     auto prefetch = [&](const Cursor& c) -> Pre {
-      Pre p{0.f, 0.f, 0.f, 0.f};
+      Pre p{0u, 0.f, 0.f, 0.f};
       if (!c.valid) return p;
       const int len = min(kTile, c.U.len - c.jt * kTile);
-      if (r < len) p.dt = load_f(kp.dt, (c.U.start + (int64_t)c.jt * kTile + r) * g.H + c.U.h, 1);
+      if (r < len)
+        p.dt = ld_global_u16(reinterpret_cast<const __nv_bfloat16*>(kp.dt) +
+                             (c.U.start + (int64_t)c.jt * kTile + r) * g.H + c.U.h);
       p.A = kp.A[c.U.h];
       p.bias = kp.dt_bias ? kp.dt_bias[c.U.h] : 0.f;
       p.D = kp.D ? kp.D[c.U.h] : 0.f;
@@ -730,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float la = 0.f;
       dl = 0.f;
       if (r < len) {
-        dl = softplus_f(p.dt + p.bias);
+        dl = softplus_f(__uint_as_float(p.dt << 16) + p.bias);
         la = dl * p.A * LOG2E;
       }
       cs = la;
@@ -926,11 +755,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
+namespace tc {
+namespace {
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
@@ -943,9 +771,10 @@ EncodeTiledFn encode_fn() {
   }
   return fn;
 }
+}  // namespace
 
-bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+bool encode_bf16_sw128(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                       const cuuint64_t* strides_bytes, const cuuint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t es[3] = {1, 1, 1};
@@ -953,8 +782,7 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
             box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
+}  // namespace tc
 
 bool tc_supported(const Geom& g, const Args*) {
   if (!g.in_bf16 || !g.out_bf16) return false;
@@ -971,21 +799,22 @@ int tc_kernels(const Geom&) { return 1; }
 size_t tc_workspace_bytes(const Geom&) { return 256; }
 
 cudaError_t tc_forward(const Geom& g, const Args& a, void*, int* status, cudaStream_t stream,
-                       int num_sms) {
+                       int num_sms, int unit_columns) {
+  if (unit_columns == 128) return tc_wide_forward(g, a, status, stream, num_sms);
   CUtensorMap tx, tb, tc;
   const cuuint64_t T = (cuuint64_t)g.tokens;
   {
     cuuint64_t dims[2] = {(cuuint64_t)g.H * g.P, T};
     cuuint64_t str[1] = {(cuuint64_t)g.H * g.P * 2};
     cuuint32_t box[2] = {64, kTile};
-    if (!encode(&tx, a.x, 2, dims, str, box)) return cudaErrorInvalidValue;
+    if (!tc::encode_bf16_sw128(&tx, a.x, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   {
     cuuint64_t dims[3] = {(cuuint64_t)g.N, (cuuint64_t)g.G, T};
     cuuint64_t str[2] = {(cuuint64_t)g.N * 2, (cuuint64_t)g.G * g.N * 2};
     cuuint32_t box[3] = {64, 1, kTile};
-    if (!encode(&tb, a.B, 3, dims, str, box)) return cudaErrorInvalidValue;
-    if (!encode(&tc, a.C, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!tc::encode_bf16_sw128(&tb, a.B, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!tc::encode_bf16_sw128(&tc, a.C, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
   KParams kp;
   kp.g = g;

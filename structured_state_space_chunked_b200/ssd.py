@@ -20,6 +20,7 @@ _lib = None
 SSD_F32, SSD_BF16 = 0, 1
 SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_TC = -1, 0, 1
 SSD_OPT_FORCE_PATH = 1
+SSD_OPT_TC_UNIT_COLUMNS = 2
 ERRORS = {
     0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3: "SSD_ERR_CUDA",
     -4: "SSD_ERR_TIMEOUT", -5: "SSD_ERR_OOM", -6: "SSD_ERR_BAD_SEQLENS",
@@ -153,6 +154,12 @@ class SSD:
     # -- options ---------------------------------------------------------------------
     def force_path(self, path: int) -> None:
         rc = lib().ssd_set_option(self._h, SSD_OPT_FORCE_PATH, int(path))
+        if rc:
+            raise SSDError(rc, "ssd_set_option")
+
+    def tc_unit_columns(self, cols: int) -> None:
+        """Column width (64 or 128) of the tensor-core kernel's work units."""
+        rc = lib().ssd_set_option(self._h, SSD_OPT_TC_UNIT_COLUMNS, int(cols))
         if rc:
             raise SSDError(rc, "ssd_set_option")
 

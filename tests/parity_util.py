@@ -26,7 +26,7 @@ def to_np(t):
     return t.detach().to("cpu").double().numpy()
 
 
-def gpu_run(w, inp, path=ssd.SSD_PATH_AUTO, chunk_size=None, handle=None):
+def gpu_run(w, inp, path=ssd.SSD_PATH_AUTO, chunk_size=None, handle=None, unit_columns=None):
     """Run the CUDA path through the C ABI; inputs already on the device."""
     max_docs = 0 if inp["cu_seqlens"] is None else inp["cu_seqlens"].numel() - 1
     bsz, L = inp["x"].shape[:2]
@@ -34,6 +34,8 @@ def gpu_run(w, inp, path=ssd.SSD_PATH_AUTO, chunk_size=None, handle=None):
                           max_docs=max_docs)
     if path != ssd.SSD_PATH_AUTO:
         h.force_path(path)
+    if unit_columns is not None:
+        h.tc_unit_columns(unit_columns)
     y, fin = h.forward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
                        inp["dt_bias"], chunk_size or w.chunk_size, inp["initial_states"],
                        inp["cu_seqlens"])

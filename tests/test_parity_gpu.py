@@ -34,6 +34,9 @@ SMALL = [
     ("bf16", 1, 333, 4, 128, 128, 4, 128, "normal0.1"),
     ("bf16", 1, 290, 2, 128, 256, 1, 256, "normal0.1"),
     ("bf16", 3, 129, 2, 64, 128, 2, 128, "normal0.1"),
+    ("bf16", 1, 200, 2, 256, 128, 1, 128, "normal0.1"),
+    ("bf16", 2, 250, 4, 64, 64, 2, 256, "normal0.1"),
+    ("bf16", 1, 140, 2, 64, 32, 1, 128, "zero"),
 ]
 
 
@@ -47,6 +50,42 @@ def test_small_shapes(case, path):
     inp = make(w)
     y, fin, _ = gpu_run(w, inp, path)
     check(w, inp, y, fin)
+
+
+def _wide_ok(w):
+    # 128-column units: N <= 128 and whole units in one B/C group
+    if w.dtype != "bf16" or w.dstate > 128 or w.chunk_size % 128:
+        return False
+    if w.headdim % 128 == 0:
+        return w.headdim <= 256
+    return w.headdim == 64 and (w.nheads // w.ngroups) % 2 == 0
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "-".join(map(str, c)))
+def test_small_shapes_128_column_units(case):
+    dtype, b, L, H, P, N, G, Q, init = case
+    w = I.random_small(7 + L, dtype, b, L, H, P, N, G, Q, init)
+    if not _wide_ok(w):
+        pytest.skip("shape outside 128-column units")
+    inp = make(w)
+    y, fin, _ = gpu_run(w, inp, ssd.SSD_PATH_TC, unit_columns=128)
+    check(w, inp, y, fin)
+
+
+@pytest.mark.parametrize("name", ["mamba2_130m_layer_b4_L2048", "varlen_32k_H32_P64_N128",
+                                  "long_L2048_H64_P128_N128_G8"])
+def test_workloads_128_column_units_sampled(name):
+    w = I.workload(name)
+    inp = make(w)
+    y, fin, _ = gpu_run(w, inp, ssd.SSD_PATH_TC, unit_columns=128)
+    check(w, inp, y, fin, heads=[0, 1, w.nheads - 1])
+
+
+def test_128_column_units_unsupported_shape_is_refused():
+    w = I.random_small(3, "bf16", 1, 256, 3, 64, 128, 3, 128, "zero")  # H/G = 1: no head pair
+    inp = make(w)
+    with pytest.raises(ssd.SSDError):
+        gpu_run(w, inp, ssd.SSD_PATH_TC, unit_columns=128)
 
 
 @pytest.mark.parametrize("Q", [1, 3, 16, 64, 100, 128, 256])
