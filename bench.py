@@ -205,6 +205,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--unit-columns", type=int, default=64, choices=[64, 128],
+                    help="column width of the tensor-core kernel's work units")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     args = ap.parse_args()
@@ -266,8 +268,12 @@ def main():
     path = {"auto": ssd.SSD_PATH_AUTO, "simt": ssd.SSD_PATH_SIMT, "tc": ssd.SSD_PATH_TC}[args.path]
     if path != ssd.SSD_PATH_AUTO:
         h.force_path(path)
+    if args.unit_columns != 64:
+        h.tc_unit_columns(args.unit_columns)
     plan = h.plan(w.chunk_size, ndocs if inp["cu_seqlens"] is not None else 0)
     path_name = {0: "simt", 1: "tc"}[plan.path if path == ssd.SSD_PATH_AUTO else path]
+    if path_name == "tc" and args.unit_columns == 128:
+        path_name = "tc128"
     y = torch.empty_like(inp["x"])
     fin = torch.empty(ndocs, w.nheads, w.dstate, w.headdim, dtype=torch.float32, device=dev)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -326,7 +332,8 @@ def main():
                  else "fallback", "algorithmic_bytes_per_launch": byts,
                  "causal_flops_per_launch": flops, "tensor_tflops_achieved": achieved_tf,
                  "roofline_us": 1e6 * max(t_hbm, t_tc), "frac_of_roofline": 1e3 * max(t_hbm, t_tc) / ms,
-                 "kernel": traffic_kernel or ("ssd_tc_fused" if path_name == "tc" else "simt (4-5 kernels)")})
+                 "kernel": traffic_kernel or {"tc": "ssd_tc_fused", "tc128": "ssd_tc_wide"}.get(
+                     path_name, "simt (4-5 kernels)")})
 
     # end to end through the host-buffer entry point (pinned host memory)
     host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in inp.items()}
