@@ -211,6 +211,33 @@ def test_empty_sequence_and_null_optionals():
     assert torch.equal(fin, init)
 
 
+@pytest.mark.parametrize("case", [
+    # dtype, batch, seqlen, H, P, N, G, Q, varlen lengths (None: batch mode), pinned
+    ("bf16", 9, 200, 4, 64, 128, 1, 256, None, True),
+    ("bf16", 1, 0, 4, 64, 128, 1, 128, [1, 0, 300, 17, 0, 1, 129, 128, 2, 40, 260], False),
+    ("bf16", 1, 0, 4, 64, 128, 1, 128, [700], True),
+    ("fp32", 3, 150, 2, 32, 16, 1, 64, None, False),
+], ids=["batch9-pinned", "varlen11", "one-doc", "fp32-batch3"])
+def test_host_entry_point_pipelined_equals_device_call(case):
+    # ssd_forward_host splits the documents into groups whose copies and compute
+    # overlap; every group computes the same units as one device call
+    dtype, b, L, H, P, N, G, Q, lens, pinned = case
+    cu = None
+    if lens is not None:
+        cu = I.cu_seqlens_from_lengths(lens)
+        L = int(cu[-1])
+    w = I.random_small(31 + L, dtype, b, L, H, P, N, G, Q, "normal0.1",
+                       varlen_tokens=L if lens is not None else 0)
+    inp = make(w, cu_seqlens=cu)
+    y1, f1, h = gpu_run(w, inp)
+    host = {k: (None if v is None else (v.cpu().pin_memory() if pinned else v.cpu()))
+            for k, v in inp.items()}
+    yh, fh = h.forward_host(host["x"], host["dt"], host["A"], host["B"], host["C"], host["D"],
+                            host["dt_bias"], Q, host["initial_states"], host["cu_seqlens"])
+    assert h.status() == 0
+    assert torch.equal(yh, y1.cpu()) and torch.equal(fh, f1.cpu())
+
+
 def test_deterministic_and_host_entry_point_agree():
     w = I.random_small(12, "bf16", 2, 300, 4, 64, 128, 1, 256, "normal0.1")
     inp = make(w)
