@@ -57,13 +57,22 @@ def algorithmic(w, ndocs):
     return byts, T * H * flops_tok_head
 
 
-def kernel_source_hash():
+# the sources each measured kernel is built from (its recorded DRAM traffic stays
+# valid while these are unchanged)
+KERNEL_SOURCES = {
+    "tc": ("ssd_tc.cu", "tc_common.cuh", "ssd_internal.h"),
+    "tc128": ("ssd_tc_wide.cu", "tc_common.cuh", "ssd_internal.h"),
+    "simt": ("ssd_simt.cu", "ssd_internal.h"),
+    "step": ("ssd_step.cu", "ssd_internal.h"),
+}
+
+
+def kernel_source_hash(path_name="tc"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "structured_state_space_chunked_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(f.read())
+    for fn in KERNEL_SOURCES[path_name]:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -74,7 +83,7 @@ def recorded_traffic(workload, path_name):
         with open(fn) as f:
             rec = json.load(f)
         e = rec[workload][path_name]
-        if e.get("source_hash") == kernel_source_hash():
+        if e.get("source_hash") == kernel_source_hash(path_name):
             return float(e["dram_bytes_per_launch"]), e.get("kernel")
     except Exception:
         pass
@@ -197,6 +206,103 @@ def oracle_sample_throughput(w, inp, budget_s):
 
 
 # ----------------------------------------------------------------------------- main
+def run_step(args, w, rank, world, local, pg, hbm_peak, peak_kind):
+    """--op step: ``ssd_step`` over a decode batch with the workload's head shape.
+
+    A step reads and writes every sequence's fp32 state (8 N P bytes per head) plus
+    the token's x, dt, B, C and y; that is its compulsory traffic and the kernel is
+    HBM-bound.  The state is updated in place, step after step; L2 is flushed before
+    every timed step.
+    """
+    import math
+    import numpy as np
+    import torch
+
+    from structured_state_space_chunked_b200 import ssd
+
+    dev = torch.device("cuda", local)
+    bsz, H, P, N, G = args.decode_batch, w.nheads, w.headdim, w.dstate, w.ngroups
+    td = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    g = torch.Generator(device="cpu").manual_seed(1234 + rank)
+    x = torch.randn(bsz, H, P, generator=g).to(dev, td)
+    dt = torch.randn(bsz, H, generator=g).to(dev, td)
+    A = (-torch.exp(torch.rand(H, generator=g) * math.log(16))).to(dev)
+    B = (torch.randn(bsz, G, N, generator=g) / math.sqrt(N)).to(dev, td)
+    C = (torch.randn(bsz, G, N, generator=g) / math.sqrt(N)).to(dev, td)
+    D = torch.randn(H, generator=g).to(dev)
+    u = torch.exp(torch.rand(H, generator=g) * (math.log(1e-1) - math.log(1e-3)) + math.log(1e-3))
+    bias = torch.log(torch.expm1(u)).to(dev)
+    state = (0.1 * torch.randn(bsz, H, N, P, generator=g)).to(dev)
+    y = torch.empty(bsz, H, P, dtype=td, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ssd.ssd_step(x, dt, A, B, C, state, D, bias, y=y)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.2)
+    barrier(pg)
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    barrier(pg)
+    t_wall1 = time.time()
+    clk.region(t_wall0, t_wall1)
+    time.sleep(0.1)
+    clocks = clk.stop()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    ms = max_over_ranks(pg, ms)
+    ein = 2 if w.dtype == "bf16" else 4
+    byts = bsz * H * (8 * N * P + 2 * P * ein + ein) + 2 * bsz * G * N * ein + 12 * H
+    achieved = byts / (ms * 1e-3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        nb = min(bsz, 32)
+        args_cpu = [t[:nb].cpu() for t in (state, x, dt)] + [A.cpu()] + [t[:nb].cpu() for t in (B, C)]
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < 2.0:
+            oracle.oracle_step(*args_cpu, D.cpu(), bias.cpu())
+            reps += 1
+        dtc = (time.perf_counter() - t0) / reps
+        cpu = {"value": nb / dtc / 1e6, "unit": "Mtokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"float64 numpy step oracle, {nb} of {bsz} sequences, {reps} repetitions"}
+    if rank == 0:
+        line = {
+            "metric": "SSD decode step (ssd_step) Mtokens/s and % of HBM roofline",
+            "value": bsz * world / (ms * 1e-3) / 1e6, "unit": "Mtokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": f"decode step, {w.name} head shape", "decode_batch": bsz,
+                       "nheads": H, "headdim": P, "dstate": N, "ngroups": G,
+                       "parallelism": f"dp{world} (independent replicas)",
+                       "l2": "flushed before every timed step (512 MiB write, outside the events)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak,
+                         "traffic": recorded_traffic(f"decode_b{bsz}_{w.name}", "step")[0],
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == "measured"
+                         else "fallback", "algorithmic_bytes_per_launch": byts,
+                         "kernel": "ssd_step_kernel"},
+            "cpu_baseline": cpu, "e2e": None, "gpu_launches": args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -209,6 +315,11 @@ def main():
                     help="column width of the tensor-core kernel's work units")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--op", default="forward", choices=["forward", "step"],
+                    help="forward: the chunked scan (default); step: one decode token per "
+                         "sequence (ssd_step) with the workload's head shape")
+    ap.add_argument("--decode-batch", type=int, default=256,
+                    help="sequences per ssd_step call (--op step)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -220,6 +331,9 @@ def main():
     w = I.workload(args.workload)
     rank, world, local, pg = dist_setup(args.gpus)
     hbm_peak, tc_peak, peak_kind = peaks()
+    if args.op == "step":
+        run_step(args, w, rank, world, local, pg, hbm_peak, peak_kind)
+        return
 
     if args.impl == "reference":
         if rank != 0:

@@ -205,6 +205,33 @@ SSD_API int ssd_get_status(ssd_handle_t h, ssd_stream_t stream);
 SSD_API int ssd_destroy(ssd_handle_t h);
 
 /*
+ * ssd_step: one token of the recurrence for every sequence of a decode batch
+ * ("Transformers are SSMs", paperlayer.ai summary: the recurrent, linear-time
+ * mode of the selective SSM, §3.4.1, used to generate one token at a time; A is
+ * a scalar times the identity, §2.4):
+ *
+ *   delta = softplus(dt + dt_bias[h]);  S <- exp(delta A[h]) S + delta B^T x;  y = C S + D[h] x
+ *
+ *   desc      batch = number of sequences, seqlen = 1, max_docs = 0; nheads,
+ *             headdim (a multiple of 4, at most 1024), dstate, ngroups and the
+ *             dtypes as for ssd_forward.
+ *   x         [batch, H, P]  in_dtype      dt    [batch, H]  in_dtype
+ *   A         [H] fp32 (required)          D, dt_bias [H] fp32, nullable (zero)
+ *   B, C      [batch, G, N]  in_dtype (head h reads group h / (H/G))
+ *   state     [batch, H, N, P] fp32, 16-byte aligned; read and updated in place:
+ *             on return (in stream order) it holds the state after this token, so
+ *             a prefill's final_states can be passed straight in
+ *   y         [batch, H, P]  out_dtype
+ * Device pointers, owned by the caller; asynchronous on `stream`; no handle and
+ * no workspace.  SSD_ERR_INVALID_ARG for bad sizes, pointers or alignment,
+ * SSD_ERR_UNSUPPORTED for a headdim the kernel does not take.  The step moves
+ * 8 N P bytes of state per (sequence, head) and is bound by HBM bandwidth.
+ */
+SSD_API int ssd_step(const ssd_desc_t* desc, const void* x, const void* dt, const float* A,
+                     const void* B, const void* C, const float* D, const float* dt_bias,
+                     float* state, void* y, ssd_stream_t stream);
+
+/*
  * ssd_forward_noalloc: ssd_forward for callers that may not allocate device memory.
  * The paper has no counterpart to this entry point; it exists for deployment.
  *

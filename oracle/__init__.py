@@ -11,4 +11,4 @@ run as a sequential recurrence ("Transformers are SSMs", paperlayer.ai summary,
 none is "parity unpinned".
 """
 
-from .oracle import build, oracle_forward, oracle_threads  # noqa: F401
+from .oracle import build, oracle_forward, oracle_step, oracle_threads  # noqa: F401

@@ -113,3 +113,31 @@ def oracle_forward(x, dt, A, B, C, D=None, dt_bias=None, initial_states=None,
     if rc != 0:
         raise ValueError("ssd_oracle_forward rejected its arguments")
     return y.reshape(bsz, L, H, P), final
+
+
+def oracle_step(state, x, dt, A, B, C, D=None, dt_bias=None):
+    """One token of the recurrence for every sequence of a decode batch, in float64.
+
+    The same definition as ``oracle_forward`` run for a single token from a given
+    state: the recurrent (linear) mode of the selective SSM ("Transformers are
+    SSMs", paperlayer.ai summary, §3.4.1; scalar-times-identity A, §2.4).
+    Shapes: state [b,H,N,P], x [b,H,P], dt [b,H], B/C [b,G,N].  Returns
+    ``(y [b,H,P] f64, new_state [b,H,N,P] f64)``.
+    """
+    s = _f64(state)
+    x = _f64(x)
+    dt = _f64(dt)
+    A = _f64(A)
+    B = _f64(B)
+    C = _f64(C)
+    bsz, H, N, P = s.shape
+    G = B.shape[1]
+    D = np.zeros(H) if D is None else _f64(D)
+    bias = np.zeros(H) if dt_bias is None else _f64(dt_bias)
+    g = np.arange(H) // (H // G)                      # contiguous group of each head
+    delta = np.logaddexp(0.0, dt + bias[None, :])      # softplus
+    decay = np.exp(delta * A[None, :])                 # [b, H]
+    Bh, Ch = B[:, g, :], C[:, g, :]                    # [b, H, N]
+    new = decay[:, :, None, None] * s + (delta[:, :, None, None] * Bh[:, :, :, None]) * x[:, :, None, :]
+    y = np.einsum("bhn,bhnp->bhp", Ch, new) + D[None, :, None] * x
+    return y, new

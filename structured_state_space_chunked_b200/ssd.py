@@ -32,7 +32,7 @@ NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 ABI_SYMBOLS = (
     "ssd_validate_desc", "ssd_plan", "ssd_create", "ssd_set_option", "ssd_forward",
     "ssd_forward_host", "ssd_get_status", "ssd_destroy", "ssd_error_string", "ssd_version",
-    "ssd_forward_noalloc",
+    "ssd_forward_noalloc", "ssd_step",
 )
 
 
@@ -83,6 +83,8 @@ def lib():
         L.ssd_forward_noalloc.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp, vp, i32,
                                           vp, vp, i32, vp, vp, vp, vp]
         L.ssd_forward_noalloc.restype = ctypes.c_int
+        L.ssd_step.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.ssd_step.restype = ctypes.c_int
         L.ssd_destroy.argtypes = [vp]
         L.ssd_error_string.argtypes = [i32]
         L.ssd_error_string.restype = ctypes.c_char_p
@@ -281,3 +283,29 @@ def ssd_forward(x, dt, A, B, C, D=None, dt_bias=None, chunk_size=256, initial_st
         _cache[key] = h
     return h.forward(x, dt, A, B, C, D, dt_bias, chunk_size, initial_states, cu_seqlens,
                      return_final_states=return_final_states, stream=stream)
+
+
+def ssd_step(x, dt, A, B, C, state, D=None, dt_bias=None, y=None, out_dtype=None, stream=None):
+    """``ssd_step``: one decode token for every sequence, the state updated in place.
+
+    x [b,H,P], dt [b,H], B/C [b,G,N] (bf16 or fp32, one dtype), A/D/dt_bias [H] fp32,
+    state [b,H,N,P] fp32 (read and overwritten).  Returns y [b,H,P] in ``out_dtype``
+    (default: x's dtype).
+    """
+    bsz, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    if tuple(state.shape) != (bsz, H, N, P) or state.dtype != torch.float32:
+        raise ValueError(f"state must be float32 {(bsz, H, N, P)}")
+    for name, t in (("x", x), ("dt", dt), ("B", B), ("C", C), ("state", state)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    out_dtype = out_dtype or x.dtype
+    if y is None:
+        y = torch.empty(bsz, H, P, dtype=out_dtype, device=x.device)
+    desc = make_desc(bsz, 1, H, P, N, G, x.dtype, out_dtype, 0)
+    with torch.cuda.device(x.device):
+        rc = lib().ssd_step(ctypes.byref(desc), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                            _ptr(D), _ptr(dt_bias), _ptr(state), _ptr(y), _stream_ptr(stream))
+    if rc:
+        raise SSDError(rc, "ssd_step")
+    return y

@@ -107,3 +107,17 @@ def test_null_handle_and_missing_device_are_errors_not_crashes(L):
         h = vp()
         rc = L.ssd_create(ctypes.byref(_desc()), ctypes.byref(h))
         assert rc == -3 and not h.value
+
+
+def test_step_validates_its_arguments_without_a_gpu():
+    # ssd_step checks the descriptor before it touches the device
+    L = ssd.lib()
+    bad_len = ssd.make_desc(4, 2, 4, 64, 128, 1, torch.bfloat16)      # seqlen must be 1
+    bad_p = ssd.make_desc(4, 1, 4, 6, 128, 1, torch.bfloat16)         # headdim % 4
+    bad_g = ssd.make_desc(4, 1, 3, 64, 128, 2, torch.bfloat16)        # H % G
+    empty = ssd.make_desc(0, 1, 4, 64, 128, 1, torch.bfloat16)        # no sequences: nothing to do
+    null = [None] * 9
+    assert L.ssd_step(ctypes.byref(bad_len), *null, None) == -1  # SSD_ERR_INVALID_ARG
+    assert L.ssd_step(ctypes.byref(bad_p), *null, None) == -2  # SSD_ERR_UNSUPPORTED
+    assert L.ssd_step(ctypes.byref(bad_g), *null, None) == -1  # SSD_ERR_INVALID_ARG
+    assert L.ssd_step(ctypes.byref(empty), *null, None) == 0

@@ -229,3 +229,36 @@ def test_oracle_rejects_inconsistent_documents():
         oracle.oracle_forward(x, dt, A, Bm, Cm, D, bias, cu_seqlens=[0, 6, 4, 10])
     with pytest.raises(ValueError):
         oracle.oracle_forward(x, dt, A, Bm, Cm, D, bias, cu_seqlens=[0, 9])
+
+
+@pytest.mark.parametrize("seed,G,H", [(21, 1, 3), (22, 2, 4)])
+def test_decode_step_equals_the_sequential_recurrence(seed, G, H):
+    # stepping token by token from an initial state gives the recurrence run by the
+    # C oracle over the same sequence (outputs and final state)
+    b, L = 3, 9
+    x, dt, A, Bm, Cm, D, bias, init = _rand(seed, b, L, H, 5, 4, G, ndoc_init=b)
+    y_ref, fin_ref = oracle.oracle_forward(x, dt, A, Bm, Cm, D, bias, init)
+    state = init.copy()
+    ys = []
+    for t in range(L):
+        y, state = oracle.oracle_step(state, x[:, t], dt[:, t], A, Bm[:, t], Cm[:, t], D, bias)
+        ys.append(y)
+    assert _rel(np.stack(ys, axis=1), y_ref) < RTOL
+    assert _rel(state, fin_ref) < RTOL
+
+
+def test_decode_step_from_zero_state_matches_quadratic_form():
+    # from a zero state the stepped outputs are the rows of the materialised dual form
+    H, P, N, L = 2, 3, 4, 11
+    x, dt, A, Bm, Cm, D, bias, _ = _rand(23, 1, L, H, P, N, 1)
+    state = np.zeros((1, H, N, P))
+    ys = []
+    for t in range(L):
+        y, state = oracle.oracle_step(state, x[:, t], dt[:, t], A, Bm[:, t], Cm[:, t], D, bias)
+        ys.append(y[0])
+    ys = np.stack(ys)  # [L, H, P]
+    for h in range(H):
+        yq, fq = quadratic_form(x[0, :, h], _delta(dt[0, :, h], bias[h]), A[h], Bm[0, :, 0],
+                                Cm[0, :, 0], D[h])
+        assert _rel(ys[:, h], yq) < RTOL
+        assert _rel(state[0, h], fq) < RTOL
