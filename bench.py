@@ -303,6 +303,103 @@ def run_step(args, w, rank, world, local, pg, hbm_peak, peak_kind):
         pg.destroy_process_group()
 
 
+def run_cp(args, w, rank, world, local, pg, hbm_peak, peak_kind):
+    """--op cp: the device steps one context-parallel rank adds to its own forward.
+
+    The workload is the rank's slice (batch mode); the rank is the last of
+    --cp-ranks, which has the longest combine.  Timed per step: ssd_cp_logdecay,
+    ssd_cp_combine, ssd_cp_correct (the all-gather between them is a collective
+    and is not part of this one-GPU measurement).  Compulsory bytes: dt read, cs
+    written and read, C read, y read and written, every rank's final state and log
+    decay read, h_in and the final state written.
+    """
+    import torch
+
+    from structured_state_space_chunked_b200 import inputs as I
+    from structured_state_space_chunked_b200 import ssd
+
+    if w.varlen_tokens:
+        raise SystemExit("--op cp takes a batch-mode workload")
+    dev = torch.device("cuda", local)
+    inp = I.make_inputs(w, device=dev)
+    R = args.cp_ranks
+    bsz, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    y = torch.randn(bsz, L, H, P, device=dev).to(w.torch_dtype)
+    S_all = 0.1 * torch.randn(R, bsz, H, N, P, device=dev)
+    ld_all = -torch.rand(R, bsz, H, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    corr_ev = []
+
+    def step(i=None):
+        cs, ld = ssd.cp_logdecay(inp["dt"], inp["A"], inp["dt_bias"], headdim=P, dstate=N, ngroups=G)
+        h_in, fin = ssd.cp_combine(R - 1, S_all, ld_all, inp["initial_states"], dt_dtype=w.torch_dtype)
+        if i is not None:
+            corr_ev[i][0].record(stream)
+        ssd.cp_correct(inp["C"], cs, h_in, y)
+        if i is not None:
+            corr_ev[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    corr_ev.extend((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps))
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.2)
+    barrier(pg)
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        step(i)
+        ends[i].record(stream)
+    barrier(pg)
+    t_wall1 = time.time()
+    clk.region(t_wall0, t_wall1)
+    time.sleep(0.1)
+    clocks = clk.stop()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    ms = max_over_ranks(pg, ms)
+    corr_ms = sum(a.elapsed_time(b) for a, b in corr_ev) / args.steps
+    on_tc = w.dtype == "bf16" and P % 64 == 0 and P <= 256 and N % 64 == 0 and N <= 256
+    ein = 2 if w.dtype == "bf16" else 4
+    T = bsz * L
+    byts = (T * H * ein + 2 * T * H * 4 + T * G * N * ein + 2 * T * H * P * ein
+            + R * bsz * H * (N * P + 1) * 4 + 2 * bsz * H * N * P * 4)
+    flops = 2.0 * T * H * N * P
+    achieved = byts / (ms * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": "SSD context-parallel rank steps (log decay, combine, correction) Mtokens/s",
+            "value": T * world / (ms * 1e-3) / 1e6, "unit": "Mtokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": f"context-parallel rank {R - 1} of {R}, slice = {w.name}",
+                       "batch": bsz, "seqlen": L, "nheads": H, "headdim": P, "dstate": N,
+                       "ngroups": G, "parallelism": f"dp{world} (independent replicas)",
+                       "l2": "flushed before every timed step (512 MiB write, outside the events)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None,
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == "measured"
+                         else "fallback", "algorithmic_bytes_per_launch": byts,
+                         "correction_us": corr_ms * 1e3,
+                         "correction_tflops_achieved": flops / (corr_ms * 1e-3) / 1e12,
+                         "kernel": "cp_logdecay_kernel + cp_combine_kernel + "
+                                   + ("cp_correct_tc_kernel" if on_tc else "cp_correct_kernel")},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": 3 * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -315,9 +412,13 @@ def main():
                     help="column width of the tensor-core kernel's work units")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--op", default="forward", choices=["forward", "step"],
+    ap.add_argument("--op", default="forward", choices=["forward", "step", "cp"],
                     help="forward: the chunked scan (default); step: one decode token per "
-                         "sequence (ssd_step) with the workload's head shape")
+                         "sequence (ssd_step) with the workload's head shape; cp: the device "
+                         "steps a context-parallel rank adds to its forward (log decay, "
+                         "combine over --cp-ranks ranks, output correction), the workload "
+                         "being the rank's slice")
+    ap.add_argument("--cp-ranks", type=int, default=4, help="ranks for --op cp")
     ap.add_argument("--decode-batch", type=int, default=256,
                     help="sequences per ssd_step call (--op step)")
     args = ap.parse_args()
@@ -333,6 +434,9 @@ def main():
     hbm_peak, tc_peak, peak_kind = peaks()
     if args.op == "step":
         run_step(args, w, rank, world, local, pg, hbm_peak, peak_kind)
+        return
+    if args.op == "cp":
+        run_cp(args, w, rank, world, local, pg, hbm_peak, peak_kind)
         return
 
     if args.impl == "reference":

@@ -232,6 +232,47 @@ SSD_API int ssd_step(const ssd_desc_t* desc, const void* x, const void* dt, cons
                      float* state, void* y, ssd_stream_t stream);
 
 /*
+ * Context-parallel forward: the three device steps of one rank.
+ *
+ * A batch of sequences is cut along the tokens into consecutive slices, one per
+ * rank ("Transformers are SSMs", paperlayer.ai summary, §8.2: a worker hands its
+ * final state to the next; the state-passing scan of §6.2, across workers).  Rank
+ * r runs ssd_forward on its slice with no initial state, then:
+ *   1. ssd_cp_logdecay: cs[b, t, h] = sum over the slice up to t of delta A, and
+ *      logdecay[b, h] = cs at the slice's last token;
+ *   2. (the caller all-gathers every rank's final state and logdecay)
+ *   3. ssd_cp_combine: H_in = the state entering the slice, by the scan
+ *      H_in(0) = init, H_in(k+1) = exp(logdecay_k) H_in(k) + S_k over ranks k < r;
+ *      and the slice's true final state exp(logdecay_r) H_in + S_r;
+ *   4. ssd_cp_correct: y[b, t, h, :] += exp(cs[b, t, h]) C[b, t, g, :] H_in[b, h]
+ *      (the left factors of the entering state, §6.2).
+ * desc describes the rank's slice in batch mode: batch rows of seqlen tokens,
+ * max_docs = 0.  Device pointers owned by the caller, fp32 unless stated,
+ * asynchronous on `stream`:
+ *   dt [batch, L, H], C [batch, L, G, N] in_dtype;  A, dt_bias [H] (dt_bias nullable)
+ *   cs [batch, L, H], logdecay [batch, H]
+ *   local_final_all [nranks, batch, H, N, P], logdecay_all [nranks, batch, H]
+ *   initial_states [batch, H, N, P] (nullable: zero), h_in and final_states
+ *   [batch, H, N, P] (either may be NULL, not both), 16-byte aligned
+ *   y [batch, L, H, P] out_dtype, read and updated (headdim a multiple of 4)
+ *   status: one device int32 (nullable), set to SSD_ERR_TIMEOUT if a wait inside the
+ *   tensor-core correction ran out (then y is incomplete); 0 is left untouched
+ * ssd_cp_correct runs on the tensor cores for bf16 C with headdim and dstate
+ * multiples of 64 up to 256, slices of at least 128 tokens and 16-byte aligned C
+ * and y, else on the CUDA cores.
+ * Errors: SSD_ERR_INVALID_ARG for bad sizes, ranks or pointers,
+ * SSD_ERR_UNSUPPORTED for shapes the kernels do not take.
+ */
+SSD_API int ssd_cp_logdecay(const ssd_desc_t* desc, const void* dt, const float* A,
+                            const float* dt_bias, float* cs, float* logdecay, ssd_stream_t stream);
+SSD_API int ssd_cp_combine(const ssd_desc_t* desc, int rank, int nranks,
+                           const float* local_final_all, const float* logdecay_all,
+                           const float* initial_states, float* h_in, float* final_states,
+                           ssd_stream_t stream);
+SSD_API int ssd_cp_correct(const ssd_desc_t* desc, const void* C, const float* cs,
+                           const float* h_in, void* y, int* status, ssd_stream_t stream);
+
+/*
  * ssd_forward_noalloc: ssd_forward for callers that may not allocate device memory.
  * The paper has no counterpart to this entry point; it exists for deployment.
  *

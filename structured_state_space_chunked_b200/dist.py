@@ -79,3 +79,60 @@ def max_over_ranks(value: float, group=None, device: Optional[torch.device] = No
                      device=device if device is not None else "cpu")
     group.all_reduce(t, op=group.ReduceOp.MAX)
     return float(t.item())
+
+
+class _CudaOps:
+    """The device steps of a context-parallel rank, on this library's kernels."""
+
+    def __init__(self, handle):
+        self.h = handle
+
+    def forward(self, x, dt, A, B, C, D, dt_bias, chunk_size):
+        return self.h.forward(x, dt, A, B, C, D, dt_bias, chunk_size, None, None)
+
+    def logdecay(self, dt, A, dt_bias, x, B):
+        from . import ssd
+        return ssd.cp_logdecay(dt, A, dt_bias, headdim=x.shape[3], dstate=B.shape[3],
+                               ngroups=B.shape[2])
+
+    def combine(self, rank, S_all, ld_all, init, dt):
+        from . import ssd
+        return ssd.cp_combine(rank, S_all, ld_all, init, dt_dtype=dt.dtype)
+
+    def correct(self, C, cs, h_in, y):
+        from . import ssd
+        return ssd.cp_correct(C, cs, h_in, y)
+
+
+def context_parallel_forward(x, dt, A, B, C, D=None, dt_bias=None, chunk_size=256,
+                             initial_states=None, group=None, handle=None, ops=None):
+    """Chunked SSD forward over a sequence whose tokens are cut across the ranks.
+
+    Every rank holds the same batch rows; rank r holds its consecutive slice of
+    the tokens (x [b, L_r, H, P], dt [b, L_r, H], B/C [b, L_r, G, N]); slices go in
+    rank order.  ``initial_states`` is the state before the whole sequence (the
+    same on every rank, or None).  Returns this rank's y and the state at the end
+    of its slice (on the last rank: the final state of the sequence).
+
+    The one exchange step is an all-gather of each rank's local final state
+    (b·H·N·P fp32) and total log decay (b·H fp32) ("Transformers are SSMs",
+    paperlayer.ai summary, §8.2); everything else runs on the rank's own data
+    through ``ops`` (default: this library's kernels on ``handle``, a
+    :class:`ssd.SSD` of the slice's shape).
+    """
+    rank = group.get_rank() if group is not None else 0
+    world = group.get_world_size() if group is not None else 1
+    ops = ops or _CudaOps(handle)
+    y, s_local = ops.forward(x, dt, A, B, C, D, dt_bias, chunk_size)
+    cs, ld = ops.logdecay(dt, A, dt_bias, x, B)
+    if group is not None and world > 1:
+        S_parts = [torch.empty_like(s_local) for _ in range(world)]
+        ld_parts = [torch.empty_like(ld) for _ in range(world)]
+        group.all_gather(S_parts, s_local.contiguous())
+        group.all_gather(ld_parts, ld.contiguous())
+        S_all, ld_all = torch.stack(S_parts), torch.stack(ld_parts)
+    else:
+        S_all, ld_all = s_local[None], ld[None]
+    h_in, final = ops.combine(rank, S_all.contiguous(), ld_all.contiguous(), initial_states, dt)
+    ops.correct(C, cs, h_in, y)
+    return y, final

@@ -32,7 +32,7 @@ NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 ABI_SYMBOLS = (
     "ssd_validate_desc", "ssd_plan", "ssd_create", "ssd_set_option", "ssd_forward",
     "ssd_forward_host", "ssd_get_status", "ssd_destroy", "ssd_error_string", "ssd_version",
-    "ssd_forward_noalloc", "ssd_step",
+    "ssd_forward_noalloc", "ssd_step", "ssd_cp_logdecay", "ssd_cp_combine", "ssd_cp_correct",
 )
 
 
@@ -85,6 +85,11 @@ def lib():
         L.ssd_forward_noalloc.restype = ctypes.c_int
         L.ssd_step.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.ssd_step.restype = ctypes.c_int
+        L.ssd_cp_logdecay.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp]
+        L.ssd_cp_combine.argtypes = [ctypes.POINTER(Desc), i32, i32, vp, vp, vp, vp, vp, vp]
+        L.ssd_cp_correct.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp]
+        for name in ("ssd_cp_logdecay", "ssd_cp_combine", "ssd_cp_correct"):
+            getattr(L, name).restype = ctypes.c_int
         L.ssd_destroy.argtypes = [vp]
         L.ssd_error_string.argtypes = [i32]
         L.ssd_error_string.restype = ctypes.c_char_p
@@ -308,4 +313,56 @@ def ssd_step(x, dt, A, B, C, state, D=None, dt_bias=None, y=None, out_dtype=None
                             _ptr(D), _ptr(dt_bias), _ptr(state), _ptr(y), _stream_ptr(stream))
     if rc:
         raise SSDError(rc, "ssd_step")
+    return y
+
+
+# -- context-parallel device steps (see include/ssd.h) -----------------------------------
+
+def _cp_desc(dt, nheads, headdim, dstate, ngroups, out_dtype):
+    bsz, L = dt.shape[0], dt.shape[1]
+    return make_desc(bsz, L, nheads, headdim, dstate, ngroups, dt.dtype, out_dtype, 0)
+
+
+def cp_logdecay(dt, A, dt_bias=None, headdim=4, dstate=1, ngroups=1, stream=None):
+    """``ssd_cp_logdecay``: (cs [b,L,H] fp32, logdecay [b,H] fp32) of this slice."""
+    bsz, L, H = dt.shape
+    cs = torch.empty(bsz, L, H, dtype=torch.float32, device=dt.device)
+    ld = torch.empty(bsz, H, dtype=torch.float32, device=dt.device)
+    desc = _cp_desc(dt, H, headdim, dstate, ngroups, dt.dtype)
+    with torch.cuda.device(dt.device):
+        rc = lib().ssd_cp_logdecay(ctypes.byref(desc), _ptr(dt), _ptr(A), _ptr(dt_bias),
+                                   _ptr(cs), _ptr(ld), _stream_ptr(stream))
+    if rc:
+        raise SSDError(rc, "ssd_cp_logdecay")
+    return cs, ld
+
+
+def cp_combine(rank, local_final_all, logdecay_all, initial_states=None, dt_dtype=torch.bfloat16,
+               stream=None):
+    """``ssd_cp_combine``: (h_in, final_state) of ``rank`` from every rank's
+    local final state [R,b,H,N,P] and log decay [R,b,H]."""
+    R, bsz, H, N, P = local_final_all.shape
+    h_in = torch.empty(bsz, H, N, P, dtype=torch.float32, device=local_final_all.device)
+    fin = torch.empty_like(h_in)
+    desc = make_desc(bsz, 1, H, P, N, 1, dt_dtype, dt_dtype, 0)
+    with torch.cuda.device(local_final_all.device):
+        rc = lib().ssd_cp_combine(ctypes.byref(desc), int(rank), int(R), _ptr(local_final_all),
+                                  _ptr(logdecay_all), _ptr(initial_states), _ptr(h_in), _ptr(fin),
+                                  _stream_ptr(stream))
+    if rc:
+        raise SSDError(rc, "ssd_cp_combine")
+    return h_in, fin
+
+
+def cp_correct(C, cs, h_in, y, status=None, stream=None):
+    """``ssd_cp_correct``: y += exp(cs) C H_in, in place.  ``status`` is an optional
+    one-element int32 device tensor that receives a device-side timeout code."""
+    bsz, L, G, N = C.shape
+    H, P = y.shape[2], y.shape[3]
+    desc = make_desc(bsz, L, H, P, N, G, C.dtype, y.dtype, 0)
+    with torch.cuda.device(y.device):
+        rc = lib().ssd_cp_correct(ctypes.byref(desc), _ptr(C), _ptr(cs), _ptr(h_in), _ptr(y),
+                                  _ptr(status), _stream_ptr(stream))
+    if rc:
+        raise SSDError(rc, "ssd_cp_correct")
     return y

@@ -92,3 +92,83 @@ def test_two_gloo_ranks_split_a_batch(tmp_path):
     assert res["equal_y"] and res["equal_f"]
     assert res["max"] == 11.0
     assert res["ranges"] == [[0, 3], [3, 5]]
+
+
+class _CpuOps:
+    """Test-only float64 stand-ins for the device steps of a context-parallel rank
+    (the collectives and their orchestration are the code under test)."""
+
+    def forward(self, x, dt, A, B, C, D, dt_bias, chunk_size):
+        import oracle
+        y, fin = oracle.oracle_forward(x, dt, A, B, C, D, dt_bias, None)
+        return torch.tensor(y), torch.tensor(fin)
+
+    def logdecay(self, dt, A, dt_bias, x, B):
+        la = np.logaddexp(0.0, dt.double().numpy() + dt_bias.double().numpy()[None, None, :])
+        cs = np.cumsum(la * A.double().numpy()[None, None, :], axis=1)
+        return torch.tensor(cs), torch.tensor(np.ascontiguousarray(cs[:, -1]))
+
+    def combine(self, rank, S_all, ld_all, init, dt):
+        S, ld = S_all.numpy(), ld_all.numpy()
+        h = np.zeros(S.shape[1:]) if init is None else init.double().numpy().copy()
+        for k in range(rank):
+            h = np.exp(ld[k])[..., None, None] * h + S[k]
+        return torch.tensor(h), torch.tensor(np.exp(ld[rank])[..., None, None] * h + S[rank])
+
+    def correct(self, C, cs, h_in, y):
+        H, G = y.shape[2], C.shape[2]
+        Ch = C.double().numpy()[:, :, np.arange(H) // (H // G), :]        # [b, L, H, N]
+        add = np.einsum("blhn,bhnp->blhp", Ch, h_in.numpy()) * np.exp(cs.numpy())[..., None]
+        y += torch.tensor(add)
+        return y
+
+
+def _cp_rank_main(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import oracle
+    from structured_state_space_chunked_b200 import dist as d
+    from structured_state_space_chunked_b200 import inputs as I
+
+    group = d.init("gloo", timeout_s=60)
+    w = I.random_small(91, "fp32", 2, 42, 4, 3, 5, 2, 16, "normal0.1")
+    inp = I.make_inputs(w)
+    t0, t1 = d.shard_range(w.seqlen, world, rank)
+    part = {k: inp[k][:, t0:t1].contiguous() for k in ("x", "dt", "B", "C")}
+    y, fin = d.context_parallel_forward(part["x"], part["dt"], inp["A"], part["B"], part["C"],
+                                        inp["D"], inp["dt_bias"], 16, inp["initial_states"],
+                                        group=group, ops=_CpuOps())
+    gathered = [None] * world
+    group.all_gather_object(gathered, (t0, t1, y.numpy().tolist(), fin.numpy().tolist()))
+    if rank == 0:
+        yf, ff = oracle.oracle_forward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                       inp["dt_bias"], inp["initial_states"])
+        ys = np.concatenate([np.asarray(g[2]) for g in gathered], axis=1)
+        ey = float(np.max(np.abs(ys - yf)) / np.max(np.abs(yf)))
+        ef = float(np.max(np.abs(np.asarray(gathered[-1][3]) - ff)) / np.max(np.abs(ff)))
+        with open(os.path.join(out_dir, "cp.json"), "w") as f:
+            json.dump(dict(ey=ey, ef=ef, ranges=[(g[0], g[1]) for g in gathered]), f)
+    group.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_parallel_ranks_reproduce_the_whole_sequence(tmp_path, world):
+    # each rank holds a slice of the tokens; after the all-gather of local final
+    # states and log decays, the ranks' outputs together equal one run over the
+    # whole sequence, and the last rank holds its final state
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_cp_rank_main, args=(r, world, port, str(tmp_path)))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = json.load(open(tmp_path / "cp.json"))
+    assert res["ey"] < 1e-10 and res["ef"] < 1e-10, res
+    assert res["ranges"][0][0] == 0 and res["ranges"][-1][1] == 42
