@@ -7,8 +7,10 @@ library never calls it and shares no code with it.
 The oracle is the plain definition of the scalar-times-identity selective SSM
 run as a sequential recurrence ("Transformers are SSMs", paperlayer.ai summary,
 §2.4, §3.4.1 and App. B.2.1), written in C (``ssd_oracle.c``) and driven from
-``oracle.py``.  Every function here is pinned by ``tests/test_oracle_pins.py``;
-none is "parity unpinned".
+``oracle.py``.  ``oracle_backward`` is the gradient of the same recurrence by the
+chain rule.  Every function here is pinned by ``tests/test_oracle_pins.py``; none
+is "parity unpinned".
 """
 
-from .oracle import build, oracle_forward, oracle_step, oracle_threads  # noqa: F401
+from .oracle import (build, oracle_backward, oracle_forward, oracle_step,  # noqa: F401
+                     oracle_threads)

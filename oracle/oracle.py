@@ -47,6 +47,18 @@ def _load():
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
         ]
+        f = lib.ssd_oracle_backward
+        f.restype = ctypes.c_int
+        f.argtypes = [
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ]
         lib.ssd_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -141,3 +153,70 @@ def oracle_step(state, x, dt, A, B, C, D=None, dt_bias=None):
     new = decay[:, :, None, None] * s + (delta[:, :, None, None] * Bh[:, :, :, None]) * x[:, :, None, :]
     y = np.einsum("bhn,bhnp->bhp", Ch, new) + D[None, :, None] * x
     return y, new
+
+
+def oracle_backward(x, dt, A, B, C, dy, D=None, dt_bias=None, initial_states=None,
+                    dfinal_states=None, cu_seqlens=None, heads=None, nthreads: int = 0):
+    """Gradient of ``sum <dy, y> + <dfinal_states, final_states>`` with respect to
+    every input of ``oracle_forward``, in float64: the chain rule taken backwards
+    through the same sequential recurrence (``ssd_oracle_backward`` in the C file
+    states each step).
+
+    Shapes as for ``oracle_forward``; ``dy`` like ``x``; ``dfinal_states`` like the
+    final states (None: zero).  ``heads`` restricts the computation to those heads:
+    their per-head gradients are filled (the others stay NaN) and dB / dC hold only
+    their share.  Returns a dict with dx, ddt, dA, dB, dC, dD, ddt_bias and
+    dinitial_states (the gradient with respect to the initial states, present
+    whether or not initial states were given)."""
+    x = _f64(x)
+    dt = _f64(dt)
+    A = _f64(A)
+    B = _f64(B)
+    C = _f64(C)
+    D = _f64(D)
+    dt_bias = _f64(dt_bias)
+    init = _f64(initial_states)
+    dy = _f64(dy)
+    dfin = _f64(dfinal_states)
+    bsz, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    T = bsz * L
+    if cu_seqlens is None:
+        offsets = np.arange(bsz + 1, dtype=np.int64) * L
+    else:
+        if bsz != 1:
+            raise ValueError("cu_seqlens requires a single packed row (batch == 1)")
+        offsets = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    ndocs = len(offsets) - 1
+    for name, a in (("initial_states", init), ("dfinal_states", dfin)):
+        if a is not None and a.shape != (ndocs, H, N, P):
+            raise ValueError(f"{name} must be {(ndocs, H, N, P)}, got {a.shape}")
+    if dy.shape != x.shape:
+        raise ValueError("dy must have the shape of x")
+    sel = None
+    if heads is not None:
+        sel = np.ascontiguousarray(np.asarray(heads, dtype=np.int32))
+    dx = np.full((T, H, P), np.nan)
+    ddt = np.full((T, H), np.nan)
+    dB = np.zeros((T, G, N))
+    dC = np.zeros((T, G, N))
+    dA_part = np.full((ndocs, H), np.nan)
+    dD_part = np.full((ndocs, H), np.nan)
+    db_part = np.full((ndocs, H), np.nan)
+    dinit = np.full((ndocs, H, N, P), np.nan)
+    rc = _load().ssd_oracle_backward(
+        T, H, P, N, G, ndocs, _ptr(offsets),
+        _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(dt_bias), _ptr(init),
+        _ptr(dy), _ptr(dfin), _ptr(sel), 0 if sel is None else len(sel),
+        _ptr(dx), _ptr(ddt), _ptr(dA_part), _ptr(dB), _ptr(dC), _ptr(dD_part), _ptr(db_part),
+        _ptr(dinit), int(nthreads),
+    )
+    if rc == -2:
+        raise MemoryError("ssd_oracle_backward ran out of host memory")
+    if rc != 0:
+        raise ValueError("ssd_oracle_backward rejected its arguments")
+    return {
+        "dx": dx.reshape(bsz, L, H, P), "ddt": ddt.reshape(bsz, L, H),
+        "dA": dA_part.sum(axis=0), "dB": dB.reshape(bsz, L, G, N), "dC": dC.reshape(bsz, L, G, N),
+        "dD": dD_part.sum(axis=0), "ddt_bias": db_part.sum(axis=0), "dinitial_states": dinit,
+    }

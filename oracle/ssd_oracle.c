@@ -132,3 +132,174 @@ int ssd_oracle_max_threads(void) {
   return 1;
 #endif
 }
+
+/*
+ * ssd_oracle_backward -- the gradient of the same recurrence, by the chain rule
+ * taken backwards through the tokens (reverse-mode differentiation of the
+ * definition above; the pages give only its cost, "Transformers are SSMs",
+ * paperlayer.ai summary, §6 and §3.4.1).  The loss is
+ *     sum_t <dy_t, y_t> + <dfinal, final_state>
+ * for given cotangents dy [T,H,P] and dfinal [ndocs,H,N,P] (NULL: zero).  With
+ * Gm the cotangent of the state S_t, walking t from the document's last token
+ * down to its first:
+ *
+ *     Gm      += C_t^T dy_t                       (y_t reads S_t)
+ *     dC_t    += S_t dy_t                         dD      += <dy_t, x_t>
+ *     gB       = Gm^T B_t                         dx_t     = delta_t gB + D dy_t
+ *     dB_t    += delta_t Gm x_t
+ *     ddelta_t = <x_t, gB> + A exp(delta_t A) <Gm, S_{t-1}>
+ *     dA      += delta_t exp(delta_t A) <Gm, S_{t-1}>
+ *     ddt_t    = ddelta_t sigmoid(dt_t + dt_bias)   ddt_bias += ddt_t
+ *     Gm       = exp(delta_t A) Gm                (cotangent of S_{t-1})
+ *
+ * and the cotangent of the initial state is Gm after the first token.  The
+ * states S_t of one (document, head) are kept from a forward sweep.  dB and dC
+ * sum over the heads of a group; dA, dD and ddt_bias come out per (document,
+ * head) in dA_part, dD_part, dbias_part [ndocs, H] (the caller sums over
+ * documents).  With a head list, only those heads are differentiated (their
+ * share of dB and dC; the other heads' entries of per-head outputs are left
+ * untouched).  dB and dC must be zero on entry.  Parallel over (document,
+ * group); the heads of a group run one after another.  Returns 0, or -1 on an
+ * inconsistent argument, or -2 when memory runs out.
+ */
+int ssd_oracle_backward(int64_t ntokens, int nheads, int headdim, int dstate, int ngroups,
+                        int ndocs, const int64_t* doc_offsets,
+                        const double* x, const double* dt, const double* A,
+                        const double* B, const double* C, const double* D,
+                        const double* dt_bias, const double* init,
+                        const double* dy, const double* dfinal,
+                        const int32_t* heads, int nheads_sel,
+                        double* dx, double* ddt, double* dA_part, double* dB, double* dC,
+                        double* dD_part, double* dbias_part, double* dinit, int nthreads) {
+  const int H = nheads, P = headdim, N = dstate, G = ngroups;
+  if (H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0 || ndocs < 0) return -1;
+  if (doc_offsets == NULL || doc_offsets[0] != 0 || doc_offsets[ndocs] != ntokens) return -1;
+  for (int d = 0; d < ndocs; ++d)
+    if (doc_offsets[d + 1] < doc_offsets[d]) return -1;
+  char* sel = (char*)calloc((size_t)H, 1);
+  if (!sel) return -2;
+  if (heads) {
+    for (int i = 0; i < nheads_sel; ++i) {
+      if (heads[i] < 0 || heads[i] >= H) {
+        free(sel);
+        return -1;
+      }
+      sel[heads[i]] = 1;
+    }
+  } else {
+    memset(sel, 1, (size_t)H);
+  }
+  const int hpg = H / G;
+  const size_t NP = (size_t)N * P;
+  const int64_t ntasks = (int64_t)ndocs * G;
+  int failed = 0;
+
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+
+#pragma omp parallel
+  {
+    int64_t maxlen = 0;
+    for (int d = 0; d < ndocs; ++d)
+      if (doc_offsets[d + 1] - doc_offsets[d] > maxlen) maxlen = doc_offsets[d + 1] - doc_offsets[d];
+    /* S[j] = state before token j of the document (S[0] = initial state) */
+    double* S = (double*)malloc(sizeof(double) * NP * (size_t)(maxlen + 1));
+    double* Gm = (double*)malloc(sizeof(double) * NP);
+    double* gB = (double*)malloc(sizeof(double) * (size_t)P);
+    if (!S || !Gm || !gB) {
+#pragma omp atomic write
+      failed = 1;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t task = 0; task < ntasks; ++task) {
+      if (!S || !Gm || !gB) continue;
+      const int d = (int)(task / G), g = (int)(task % G);
+      const int64_t t0 = doc_offsets[d], len = doc_offsets[d + 1] - t0;
+      for (int h = g * hpg; h < (g + 1) * hpg; ++h) {
+        if (!sel[h]) continue;
+        const double bias = dt_bias ? dt_bias[h] : 0.0;
+        const double skip = D ? D[h] : 0.0;
+        const size_t soff = ((size_t)d * H + h) * NP;
+        /* forward sweep, keeping every state */
+        if (init)
+          memcpy(S, init + soff, sizeof(double) * NP);
+        else
+          memset(S, 0, sizeof(double) * NP);
+        for (int64_t j = 0; j < len; ++j) {
+          const int64_t t = t0 + j;
+          const double delta = oracle_softplus(dt[t * H + h] + bias);
+          const double decay = exp(delta * A[h]);
+          const double* xt = x + ((size_t)t * H + h) * P;
+          const double* Bt = B + ((size_t)t * G + g) * N;
+          const double* prev = S + (size_t)j * NP;
+          double* next = S + (size_t)(j + 1) * NP;
+          for (int n = 0; n < N; ++n)
+            for (int p = 0; p < P; ++p)
+              next[(size_t)n * P + p] = decay * prev[(size_t)n * P + p] + delta * Bt[n] * xt[p];
+        }
+        /* backward sweep */
+        if (dfinal)
+          memcpy(Gm, dfinal + soff, sizeof(double) * NP);
+        else
+          memset(Gm, 0, sizeof(double) * NP);
+        double dA_acc = 0.0, dD_acc = 0.0, db_acc = 0.0;
+        for (int64_t j = len - 1; j >= 0; --j) {
+          const int64_t t = t0 + j;
+          const double z = dt[t * H + h] + bias;
+          const double delta = oracle_softplus(z);
+          const double decay = exp(delta * A[h]);
+          const double* xt = x + ((size_t)t * H + h) * P;
+          const double* dyt = dy + ((size_t)t * H + h) * P;
+          const double* Bt = B + ((size_t)t * G + g) * N;
+          const double* Ct = C + ((size_t)t * G + g) * N;
+          const double* St = S + (size_t)(j + 1) * NP;   /* state after token t */
+          const double* Sp = S + (size_t)j * NP;         /* state before token t */
+          double* dBt = dB + ((size_t)t * G + g) * N;
+          double* dCt = dC + ((size_t)t * G + g) * N;
+          double* dxt = dx + ((size_t)t * H + h) * P;
+          for (int n = 0; n < N; ++n)
+            for (int p = 0; p < P; ++p) Gm[(size_t)n * P + p] += Ct[n] * dyt[p];
+          for (int n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int p = 0; p < P; ++p) s += St[(size_t)n * P + p] * dyt[p];
+            dCt[n] += s;
+          }
+          for (int p = 0; p < P; ++p) dD_acc += dyt[p] * xt[p];
+          for (int p = 0; p < P; ++p) {
+            double s = 0.0;
+            for (int n = 0; n < N; ++n) s += Gm[(size_t)n * P + p] * Bt[n];
+            gB[p] = s;
+          }
+          for (int p = 0; p < P; ++p) dxt[p] = delta * gB[p] + skip * dyt[p];
+          for (int n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int p = 0; p < P; ++p) s += Gm[(size_t)n * P + p] * xt[p];
+            dBt[n] += delta * s;
+          }
+          double inner = 0.0;
+          for (size_t e = 0; e < NP; ++e) inner += Gm[e] * Sp[e];
+          double xg = 0.0;
+          for (int p = 0; p < P; ++p) xg += xt[p] * gB[p];
+          const double ddelta = xg + A[h] * decay * inner;
+          dA_acc += delta * decay * inner;
+          const double g_dt = ddelta / (1.0 + exp(-z));
+          ddt[t * H + h] = g_dt;
+          db_acc += g_dt;
+          for (size_t e = 0; e < NP; ++e) Gm[e] *= decay;
+        }
+        if (dinit) memcpy(dinit + soff, Gm, sizeof(double) * NP);
+        dA_part[(size_t)d * H + h] = dA_acc;
+        dD_part[(size_t)d * H + h] = dD_acc;
+        dbias_part[(size_t)d * H + h] = db_acc;
+      }
+    }
+    free(S);
+    free(Gm);
+    free(gB);
+  }
+  free(sel);
+  return failed ? -2 : 0;
+}

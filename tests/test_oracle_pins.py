@@ -262,3 +262,108 @@ def test_decode_step_from_zero_state_matches_quadratic_form():
                                 Cm[0, :, 0], D[h])
         assert _rel(ys[:, h], yq) < RTOL
         assert _rel(state[0, h], fq) < RTOL
+
+
+# ---- the backward oracle ------------------------------------------------------------
+# Pinned against central finite differences of oracle_forward (itself pinned above) and
+# against torch.autograd of a plain float64 loop over tokens: two independent ways of
+# differentiating the recurrence.
+
+def _bwd_case(seed, varlen):
+    r = np.random.default_rng(seed)
+    H, P, N, G = 4, 3, 2, 2
+    if varlen:
+        cu = np.array([0, 4, 4, 11, 13], dtype=np.int64)   # an empty document too
+        b, L = 1, 13
+        ndocs = 4
+    else:
+        cu = None
+        b, L = 2, 6
+        ndocs = 2
+    x, dt, A, Bm, Cm, D, bias, init = _rand(seed, b, L, H, P, N, G, ndoc_init=ndocs)
+    A = -np.exp(r.uniform(-1.0, 1.0, H))       # decays of order one: every term is visible
+    bias = r.uniform(-0.5, 0.5, H)
+    init = r.standard_normal((ndocs, H, N, P))
+    dy = r.standard_normal((b, L, H, P))
+    dfin = r.standard_normal((ndocs, H, N, P))
+    return dict(x=x, dt=dt, A=A, B=Bm, C=Cm, D=D, dt_bias=bias, initial_states=init), dy, dfin, cu
+
+
+def _loss(inp, dy, dfin, cu):
+    y, fin = oracle.oracle_forward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                   inp["dt_bias"], inp["initial_states"], cu_seqlens=cu)
+    return float(np.sum(dy * y) + np.sum(dfin * fin))
+
+
+_BWD_KEYS = [("x", "dx"), ("dt", "ddt"), ("A", "dA"), ("B", "dB"), ("C", "dC"), ("D", "dD"),
+             ("dt_bias", "ddt_bias"), ("initial_states", "dinitial_states")]
+
+
+@pytest.mark.parametrize("varlen", [False, True], ids=["batch", "packed"])
+def test_backward_equals_finite_differences_of_the_forward(varlen):
+    inp, dy, dfin, cu = _bwd_case(7, varlen)
+    g = oracle.oracle_backward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, inp["D"],
+                               inp["dt_bias"], inp["initial_states"], dfin, cu_seqlens=cu)
+    eps = 1e-6
+    for key, gkey in _BWD_KEYS:
+        base = inp[key]
+        fd = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            plus = {k: v.copy() for k, v in inp.items()}
+            minus = {k: v.copy() for k, v in inp.items()}
+            plus[key][idx] += eps
+            minus[key][idx] -= eps
+            fd[idx] = (_loss(plus, dy, dfin, cu) - _loss(minus, dy, dfin, cu)) / (2 * eps)
+        assert _rel(g[gkey], fd) < 1e-7, key
+
+
+def _torch_loss(t, dy, dfin, offsets, G):
+    """Plain float64 loop over tokens, differentiated by torch.autograd."""
+    import torch
+    x, dt, A, Bm, Cm, D, bias, init = (t[k] for k in ("x", "dt", "A", "B", "C", "D", "dt_bias",
+                                                      "initial_states"))
+    b, L, H, P = x.shape
+    xs, dts, Bs, Cs = (v.reshape(b * L, *v.shape[2:]) for v in (x, dt, Bm, Cm))
+    dys = torch.from_numpy(dy).reshape(b * L, H, P)
+    dfin_t = torch.from_numpy(dfin)
+    loss = torch.zeros((), dtype=torch.float64)
+    hpg = H // G
+    for d in range(len(offsets) - 1):
+        for h in range(H):
+            g = h // hpg
+            S = init[d, h]
+            for tok in range(offsets[d], offsets[d + 1]):
+                delta = torch.nn.functional.softplus(dts[tok, h] + bias[h])
+                S = torch.exp(delta * A[h]) * S + delta * torch.outer(Bs[tok, g], xs[tok, h])
+                y = Cs[tok, g] @ S + D[h] * xs[tok, h]
+                loss = loss + torch.dot(dys[tok, h], y)
+            loss = loss + torch.sum(dfin_t[d, h] * S)
+    return loss
+
+
+@pytest.mark.parametrize("varlen", [False, True], ids=["batch", "packed"])
+def test_backward_equals_autograd_of_a_token_loop(varlen):
+    import torch
+    inp, dy, dfin, cu = _bwd_case(11, varlen)
+    b, L = inp["x"].shape[:2]
+    offsets = list(cu) if cu is not None else [i * L for i in range(b + 1)]
+    t = {k: torch.tensor(v, dtype=torch.float64, requires_grad=True) for k, v in inp.items()}
+    _torch_loss(t, dy, dfin, offsets, inp["B"].shape[2]).backward()
+    g = oracle.oracle_backward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, inp["D"],
+                               inp["dt_bias"], inp["initial_states"], dfin, cu_seqlens=cu)
+    for key, gkey in _BWD_KEYS:
+        assert _rel(g[gkey], t[key].grad.numpy()) < 1e-12, key
+
+
+def test_backward_head_subset_matches_full_run():
+    inp, dy, dfin, cu = _bwd_case(3, False)
+    full = oracle.oracle_backward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, inp["D"],
+                                  inp["dt_bias"], inp["initial_states"], dfin)
+    part = oracle.oracle_backward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, inp["D"],
+                                  inp["dt_bias"], inp["initial_states"], dfin, heads=[1, 2])
+    for h in (1, 2):
+        assert np.array_equal(part["dx"][:, :, h], full["dx"][:, :, h])
+        assert np.array_equal(part["ddt"][:, :, h], full["ddt"][:, :, h])
+        assert np.array_equal(part["dinitial_states"][:, h], full["dinitial_states"][:, h])
+        assert part["dA"][h] == full["dA"][h]
+    assert np.isnan(part["dx"][:, :, 0]).all()
