@@ -303,6 +303,104 @@ def run_step(args, w, rank, world, local, pg, hbm_peak, peak_kind):
         pg.destroy_process_group()
 
 
+def run_bwd(args, w, rank, world, local, pg, hbm_peak, peak_kind):
+    """--op backward: ``ssd_backward`` over the workload (all gradients, fp32).
+
+    The backward runs on the CUDA cores, so its roofline is the fp32 FMA rate:
+    148 SMs x 128 lanes x 2 flops x 1965 MHz = 74.4 TFLOP/s.  Its algorithmic flops
+    per token and head, for chunks of Q = 64 tokens, are 2 Q (2 P + 3 N) (the
+    in-chunk products W, V, dC, dB, gB) + 8 N P (the state-sized products of dC, dB,
+    gB and the per-chunk cotangent sum) + 2 N P (the forward's chunk states,
+    recomputed).  L2 is flushed before every timed step.
+    """
+    import torch
+
+    from structured_state_space_chunked_b200 import inputs as I
+    from structured_state_space_chunked_b200 import ssd
+
+    dev = torch.device("cuda", local)
+    inp = I.make_inputs(w, device=dev)
+    ndocs = w.batch if inp["cu_seqlens"] is None else inp["cu_seqlens"].numel() - 1
+    dy, dfin = I.make_cotangents(w, ndocs, device=dev)
+    bsz, L = inp["x"].shape[:2]
+    H, P, N, G = w.nheads, w.headdim, w.dstate, w.ngroups
+    h = ssd.SSD(bsz, L, H, P, N, G, w.torch_dtype,
+                max_docs=0 if inp["cu_seqlens"] is None else ndocs, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return h.backward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, inp["D"],
+                          inp["dt_bias"], inp["initial_states"], dfin, inp["cu_seqlens"])
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if h.status() != 0:
+        raise SystemExit("device status set during warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.2)
+    barrier(pg)
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    barrier(pg)
+    t_wall1 = time.time()
+    clk.region(t_wall0, t_wall1)
+    time.sleep(0.1)
+    clocks = clk.stop()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    ms = max_over_ranks(pg, ms)
+    T = bsz * L
+    Q = 64
+    flops = float(T) * H * (2 * Q * (2 * P + 3 * N) + 10 * N * P)
+    peak = 148 * 128 * 2 * 1965e6 / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        heads = [0]
+        cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].cpu().numpy()
+        cpu_in = [inp[k].cpu() for k in ("x", "dt", "A", "B", "C")]
+        t0 = time.perf_counter()
+        oracle.oracle_backward(*cpu_in, dy.cpu(), inp["D"].cpu(), inp["dt_bias"].cpu(),
+                               None if inp["initial_states"] is None else inp["initial_states"].cpu(),
+                               dfin.cpu(), cu_seqlens=cu, heads=heads)
+        dtc = time.perf_counter() - t0
+        cpu = {"value": T * len(heads) / H / dtc / 1e6, "unit": "Mtokens/s",
+               "cores": min(oracle.oracle_threads(), ndocs), "kind": "oracle",
+               "sample": f"float64 backward oracle, head 0 of {H} over all {ndocs} documents, "
+                         "scaled to the whole layer"}
+    if rank == 0:
+        line = {
+            "metric": "SSD chunked-scan backward (ssd_backward) Mtokens/s and % of fp32 FMA roofline",
+            "value": T * world / (ms * 1e-3) / 1e6, "unit": "Mtokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": H,
+                       "headdim": P, "dstate": N, "ngroups": G, "input_dtype": w.dtype,
+                       "parallelism": f"dp{world} (independent replicas)",
+                       "l2": "flushed before every timed step (512 MiB write, outside the events)"},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+                         "algorithmic_flops_per_launch": flops,
+                         "kernel": "kb_chunk + kb_chunk_dstate + kb_state_pass + the forward's state kernels"},
+            "cpu_baseline": cpu, "e2e": None, "gpu_launches": 11 * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
 def run_cp(args, w, rank, world, local, pg, hbm_peak, peak_kind):
     """--op cp: the device steps one context-parallel rank adds to its own forward.
 
@@ -412,12 +510,12 @@ def main():
                     help="column width of the tensor-core kernel's work units")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--op", default="forward", choices=["forward", "step", "cp"],
+    ap.add_argument("--op", default="forward", choices=["forward", "step", "cp", "backward"],
                     help="forward: the chunked scan (default); step: one decode token per "
                          "sequence (ssd_step) with the workload's head shape; cp: the device "
                          "steps a context-parallel rank adds to its forward (log decay, "
                          "combine over --cp-ranks ranks, output correction), the workload "
-                         "being the rank's slice")
+                         "being the rank's slice; backward: ssd_backward over the workload")
     ap.add_argument("--cp-ranks", type=int, default=4, help="ranks for --op cp")
     ap.add_argument("--decode-batch", type=int, default=256,
                     help="sequences per ssd_step call (--op step)")
@@ -437,6 +535,9 @@ def main():
         return
     if args.op == "cp":
         run_cp(args, w, rank, world, local, pg, hbm_peak, peak_kind)
+        return
+    if args.op == "backward":
+        run_bwd(args, w, rank, world, local, pg, hbm_peak, peak_kind)
         return
 
     if args.impl == "reference":

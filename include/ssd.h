@@ -196,6 +196,37 @@ SSD_API int ssd_forward_host(ssd_handle_t h, const void* x, const void* dt, cons
                      int num_docs, void* y, float* final_states, ssd_stream_t stream);
 
 /*
+ * ssd_backward: the gradient of the forward pass.  The pages give only its cost
+ * ("Transformers are SSMs", paperlayer.ai summary: training FLOPs of the SSD layer,
+ * §6); what it computes is the derivative of the same recurrence, taken through
+ * the block decomposition of §6 one chunk at a time.  For the loss
+ *
+ *   sum over tokens, heads of <dy, y>  +  sum over documents, heads of <dfinal_states, final_states>
+ *
+ * it writes the gradient with respect to every input of ssd_forward.  The handle,
+ * the problem (desc, cu_seqlens, num_docs) and the inputs x, dt, A, B, C, D,
+ * dt_bias, initial_states are exactly those of the forward call being
+ * differentiated; the forward's outputs are not needed (the states are recomputed).
+ *   dy              [batch, seqlen, H, P] out_dtype (the cotangent of y; required)
+ *   dfinal_states   [docs, H, N, P] fp32 or NULL (zero)
+ * Outputs, fp32, device, owned by the caller, overwritten:
+ *   dx [batch, seqlen, H, P]; ddt [batch, seqlen, H]; dB, dC [batch, seqlen, G, N]
+ *   (summed over the heads of each group); dA [H]; dD [H] and ddt_bias [H]
+ *   (either may be NULL: not computed); dinitial_states [docs, H, N, P] or NULL.
+ * It runs on the CUDA cores in fp32 with chunks of 64 tokens whatever chunk size
+ * the forward used (the chunking changes only rounding).  dB, dC, dA, dD and
+ * ddt_bias are sums of fp32 atomic additions, so their last bits can differ from
+ * run to run.  Workspace grows in the handle as for ssd_forward.  Errors as for
+ * ssd_forward; inputs need only element alignment.
+ */
+SSD_API int ssd_backward(ssd_handle_t h, const void* x, const void* dt, const float* A,
+                         const void* B, const void* C, const float* D, const float* dt_bias,
+                         const float* initial_states, const int32_t* cu_seqlens, int num_docs,
+                         const void* dy, const float* dfinal_states, float* dx, float* ddt,
+                         float* dA, float* dB, float* dC, float* dD, float* ddt_bias,
+                         float* dinitial_states, ssd_stream_t stream);
+
+/*
  * ssd_get_status: synchronises `stream`, returns the first device-side error
  * recorded since the last call (SSD_OK if none) and clears it.
  */

@@ -8,6 +8,7 @@
 
 #include <new>
 
+#include "ssd_bwd.h"
 #include "ssd_internal.h"
 
 struct ssd_handle_s {
@@ -210,6 +211,53 @@ int ssd_forward(ssd_handle_t h, const void* x, const void* dt, const float* A, c
     ssd::simt_carve_workspace(g, h->ws, &ws);
     e = ssd::simt_forward(g, a, ws, h->status, stream);
   }
+  if (cur != h->device) cudaSetDevice(cur);
+  return cuda_rc(e);
+}
+
+int ssd_backward(ssd_handle_t h, const void* x, const void* dt, const float* A, const void* B,
+                 const void* C, const float* D, const float* dt_bias, const float* initial_states,
+                 const int32_t* cu_seqlens, int num_docs, const void* dy, const float* dfinal_states,
+                 float* dx, float* ddt, float* dA, float* dB, float* dC, float* dD, float* ddt_bias,
+                 float* dinitial_states, ssd_stream_t stream_) {
+  if (!h) return SSD_ERR_INVALID_ARG;
+  const ssd_desc_t& d = h->desc;
+  int rc = check_call(d, ssd::kBwdQ, cu_seqlens, num_docs);
+  if (rc) return rc;
+  const int64_t tokens = d.batch * d.seqlen;
+  if (tokens > 0 && (!x || !dt || !B || !C || !dy || !dx || !ddt || !dB || !dC))
+    return SSD_ERR_INVALID_ARG;
+  if (!A || !dA) return SSD_ERR_INVALID_ARG;
+  const size_t ei = elem_bytes(d.in_dtype), eo = elem_bytes(d.out_dtype);
+  if (!aligned(x, ei) || !aligned(dt, ei) || !aligned(B, ei) || !aligned(C, ei) || !aligned(dy, eo) ||
+      !aligned(A, 4) || !aligned(D, 4) || !aligned(dt_bias, 4) || !aligned(initial_states, 4) ||
+      !aligned(dfinal_states, 4) || !aligned(dx, 4) || !aligned(ddt, 4) || !aligned(dA, 4) ||
+      !aligned(dB, 4) || !aligned(dC, 4) || !aligned(dD, 4) || !aligned(ddt_bias, 4) ||
+      !aligned(dinitial_states, 4) || !aligned(cu_seqlens, 4))
+    return SSD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  Geom g;
+  make_geom(d, ssd::kBwdQ, cu_seqlens != nullptr, num_docs, &g);
+
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return SSD_ERR_CUDA;
+  const size_t need = ssd::bwd_workspace_bytes(g);
+  if (need > h->ws_bytes) {
+    if (h->ws) cudaFreeAsync(h->ws, stream);
+    h->ws = nullptr;
+    h->ws_bytes = 0;
+    cudaError_t e = cudaMallocAsync(&h->ws, need, stream);
+    if (e != cudaSuccess) {
+      h->ws = nullptr;
+      if (cur != h->device) cudaSetDevice(cur);
+      return cuda_rc(e);
+    }
+    h->ws_bytes = need;
+  }
+  ssd::Args a{x, dt, A, B, C, D, dt_bias, initial_states, cu_seqlens, nullptr, nullptr};
+  ssd::GradArgs ga{dy, dfinal_states, dx, ddt, dA, dB, dC, dD, ddt_bias, dinitial_states};
+  cudaError_t e = ssd::bwd_run(g, a, ga, h->ws, h->status, stream);
   if (cur != h->device) cudaSetDevice(cur);
   return cuda_rc(e);
 }

@@ -1,0 +1,33 @@
+// ssd_bwd.h -- declarations of the backward pass (not part of the ABI).
+#pragma once
+
+#include "ssd_internal.h"
+
+namespace ssd {
+
+// The CUDA-core forward stopped after its state pass: ws.cs, ws.delta, the state
+// entering every chunk in ws.states, and a.final_states when given (y untouched).
+cudaError_t simt_states(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
+                        cudaStream_t stream);
+
+constexpr int kBwdQ = 64;  // chunk length of the backward kernels
+
+struct GradArgs {
+  const void* dy;        // [T, H, P], out dtype
+  const float* dfinal;   // [ndocs, H, N, P] or null (zero)
+  float* dx;             // [T, H, P]
+  float* ddt;            // [T, H]
+  float* dA;             // [H]
+  float* dB;             // [T, G, N]
+  float* dC;             // [T, G, N]
+  float* dD;             // [H] or null
+  float* ddt_bias;       // [H] or null
+  float* dinit;          // [ndocs, H, N, P] or null
+};
+
+// g.Q must be kBwdQ.
+size_t bwd_workspace_bytes(const Geom& g);
+cudaError_t bwd_run(const Geom& g, const Args& a, const GradArgs& ga, void* workspace, int* status,
+                    cudaStream_t stream);
+
+}  // namespace ssd

@@ -15,39 +15,13 @@
 // table built on the device by the varlen_table kernel.
 #include <cuda_runtime.h>
 
+#include "ssd_chunks.cuh"
 #include "ssd_internal.h"
 
 namespace ssd {
 namespace {
 
 constexpr int kMaxQ = 256;
-
-struct ChunkInfo {
-  int doc;
-  int c;           // chunk index within the document
-  int64_t start;   // first token
-  int len;         // tokens in the chunk (1..Q)
-};
-
-__device__ __forceinline__ bool chunk_info(const Geom& g, const int32_t* cu,
-                                           const SimtWorkspace& ws, int64_t k, ChunkInfo* ci) {
-  if (!g.varlen) {
-    const int64_t nc = (g.seqlen + g.Q - 1) / g.Q;
-    if (nc == 0 || k >= (int64_t)g.ndocs * nc) return false;
-    ci->doc = (int)(k / nc);
-    ci->c = (int)(k % nc);
-    ci->start = (int64_t)ci->doc * g.seqlen + (int64_t)ci->c * g.Q;
-    ci->len = (int)min((int64_t)g.Q, g.seqlen - (int64_t)ci->c * g.Q);
-    return true;
-  }
-  if (!ws.total_chunks[1] || k >= ws.total_chunks[0]) return false;
-  const int d = ws.chunk_doc[k];
-  ci->doc = d;
-  ci->c = (int)(k - ws.doc_first[d]);
-  ci->start = (int64_t)cu[d] + (int64_t)ci->c * g.Q;
-  ci->len = (int)min((int64_t)g.Q, (int64_t)cu[d + 1] - ci->start);
-  return true;
-}
 
 // Inclusive block-wide sum scan (blockDim.x a multiple of 32, <= 1024).
 __device__ __forceinline__ float block_inclusive_scan(float v, float* warp_sums) {
@@ -407,8 +381,8 @@ int simt_kernels(const Geom& g) {
   return n;
 }
 
-cudaError_t simt_forward(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
-                         cudaStream_t stream) {
+cudaError_t simt_run(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
+                     cudaStream_t stream, bool outputs) {
   if (g.Q < 1 || g.Q > kMaxQ) return cudaErrorInvalidValue;
   if (g.varlen) {
     k_varlen_table<<<1, 1024, 0, stream>>>(g, a.cu, ws, status);
@@ -423,7 +397,7 @@ cudaError_t simt_forward(const Geom& g, const Args& a, const SimtWorkspace& ws, 
   if (g.ndocs > 0) {
     k_state_pass<<<dim3(g.ndocs, g.H, (unsigned)((NP + 255) / 256)), 256, 0, stream>>>(g, a, ws);
   }
-  if (g.nchunks_max > 0) {
+  if (outputs && g.nchunks_max > 0) {
     const size_t smem =
         sizeof(float) * ((size_t)kSL * (g.N + 1) + 32 * (g.N + 1) + 32 * kSP + kSL * 33 + 32 * kSP +
                          kSL + 64);
@@ -434,6 +408,16 @@ cudaError_t simt_forward(const Geom& g, const Args& a, const SimtWorkspace& ws, 
     k_chunk_scan<<<dim3((unsigned)g.nchunks_max, g.H, tiles_y), 256, smem, stream>>>(g, a, ws);
   }
   return cudaGetLastError();
+}
+
+cudaError_t simt_forward(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
+                         cudaStream_t stream) {
+  return simt_run(g, a, ws, status, stream, true);
+}
+
+cudaError_t simt_states(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
+                        cudaStream_t stream) {
+  return simt_run(g, a, ws, status, stream, false);
 }
 
 }  // namespace ssd

@@ -160,3 +160,15 @@ def random_small(seed: int, dtype: str = "bf16", batch: int = 1, seqlen: int = 3
     """A small workload with the same value recipe (parity and edge-case tests)."""
     return Workload(f"small_s{seed}", batch, seqlen, nheads, headdim, dstate, ngroups,
                     chunk_size, dtype, init, varlen_tokens, seed)
+
+
+def make_cotangents(w: Workload, ndocs: int, device="cpu", seed_offset: int = 1):
+    """Cotangents for the backward pass of ``w``: dy [b,L,H,P] in the output dtype
+    (standard normal) and dfinal_states [ndocs,H,N,P] fp32 (standard normal),
+    from their own seeded stream."""
+    rng = np.random.default_rng(w.seed + seed_offset)
+    b, L = (1, w.varlen_tokens) if w.varlen_tokens else (w.batch, w.seqlen)
+    dy = rng.standard_normal(size=(b, L, w.nheads, w.headdim), dtype=np.float32)
+    dfin = rng.standard_normal(size=(ndocs, w.nheads, w.dstate, w.headdim), dtype=np.float32)
+    return (torch.from_numpy(dy).to(w.torch_dtype).to(device),
+            torch.from_numpy(dfin).to(device))

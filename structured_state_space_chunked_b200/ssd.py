@@ -33,6 +33,7 @@ ABI_SYMBOLS = (
     "ssd_validate_desc", "ssd_plan", "ssd_create", "ssd_set_option", "ssd_forward",
     "ssd_forward_host", "ssd_get_status", "ssd_destroy", "ssd_error_string", "ssd_version",
     "ssd_forward_noalloc", "ssd_step", "ssd_cp_logdecay", "ssd_cp_combine", "ssd_cp_correct",
+    "ssd_backward",
 )
 
 
@@ -79,6 +80,8 @@ def lib():
         fwd = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, vp]
         L.ssd_forward.argtypes = fwd
         L.ssd_forward_host.argtypes = fwd
+        L.ssd_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp,
+                                   vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.ssd_get_status.argtypes = [vp, vp]
         L.ssd_forward_noalloc.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp, vp, i32,
                                           vp, vp, i32, vp, vp, vp, vp]
@@ -234,6 +237,31 @@ class SSD:
         if rc:
             raise SSDError(rc, "ssd_forward")
         return y, final_states
+
+    def backward(self, x, dt, A, B, C, dy, D=None, dt_bias=None, initial_states=None,
+                 dfinal_states=None, cu_seqlens=None, num_docs=None, stream=None):
+        """Enqueue ``ssd_backward``: the gradient of sum <dy, y> + <dfinal_states,
+        final_states> for the forward call with the same inputs.  Returns a dict of
+        fp32 tensors: dx, ddt, dA, dB, dC, dD, ddt_bias, dinitial_states."""
+        ndocs, _, _ = self._prepare(x, dt, A, B, C, D, dt_bias, initial_states, cu_seqlens,
+                                    num_docs, dy, None, False, True)
+        s = self._shapes(ndocs)
+        self._check("dfinal_states", dfinal_states, s["state"], torch.float32)
+        f32 = dict(dtype=torch.float32, device=self.device)
+        H = self.desc.nheads
+        g = {"dx": torch.empty(s["x"], **f32), "ddt": torch.empty(s["dt"], **f32),
+             "dA": torch.empty(H, **f32), "dB": torch.empty(s["B"], **f32),
+             "dC": torch.empty(s["B"], **f32), "dD": torch.empty(H, **f32),
+             "ddt_bias": torch.empty(H, **f32), "dinitial_states": torch.empty(s["state"], **f32)}
+        rc = lib().ssd_backward(self._h, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(dt_bias), _ptr(initial_states), _ptr(cu_seqlens),
+                                int(ndocs if cu_seqlens is not None else 0), _ptr(dy),
+                                _ptr(dfinal_states), _ptr(g["dx"]), _ptr(g["ddt"]), _ptr(g["dA"]),
+                                _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["ddt_bias"]),
+                                _ptr(g["dinitial_states"]), _stream_ptr(stream))
+        if rc:
+            raise SSDError(rc, "ssd_backward")
+        return g
 
     def forward_host(self, x, dt, A, B, C, D=None, dt_bias=None, chunk_size=256,
                      initial_states=None, cu_seqlens=None, num_docs=None, y=None,

@@ -121,3 +121,9 @@ def test_step_validates_its_arguments_without_a_gpu():
     assert L.ssd_step(ctypes.byref(bad_p), *null, None) == -2  # SSD_ERR_UNSUPPORTED
     assert L.ssd_step(ctypes.byref(bad_g), *null, None) == -1  # SSD_ERR_INVALID_ARG
     assert L.ssd_step(ctypes.byref(empty), *null, None) == 0
+
+
+def test_backward_refuses_a_missing_handle_without_a_gpu():
+    # ssd_backward checks its handle before it touches the device
+    L = ssd.lib()
+    assert L.ssd_backward(None, *([None] * 9), 0, *([None] * 11)) == -1  # SSD_ERR_INVALID_ARG
