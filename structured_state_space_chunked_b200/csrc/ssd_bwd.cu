@@ -35,7 +35,7 @@
 namespace ssd {
 namespace {
 
-constexpr int kLD = 65;            // padded row stride of the 64 x 64 shared tiles
+constexpr int kLD = 68;            // row stride of the 64 x 64 shared tiles (16-byte rows)
 constexpr int kTileF = 64 * kLD;   // floats per tile
 
 struct BwdWs {
@@ -115,7 +115,24 @@ __global__ void __launch_bounds__(256) kb_state_pass(Geom g, Args a, GradArgs ga
   const int64_t cnt = doc_chunks(g, ws, d, &first);
   const int64_t so = ((int64_t)d * g.H + h) * NP + e;
   float carry = ga.dfinal ? ga.dfinal[so] : 0.f;
-  for (int64_t c = cnt - 1; c >= 0; --c) {
+  // eight chunks per round: their loads are all issued before the dependent updates
+  constexpr int kU = 8;
+  int64_t c = cnt - 1;
+  for (; c + 1 >= kU; c -= kU) {
+    float s[kU], dec[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t kk = first + c - u;
+      s[u] = bw.dstates[(kk * g.H + h) * NP + e];
+      dec[u] = ws.cs[((int64_t)h * g.nchunks_max + kk) * g.Q + g.Q - 1];
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      bw.dstates[((first + c - u) * g.H + h) * NP + e] = carry;
+      carry = fmaf(expf(dec[u]), carry, s[u]);
+    }
+  }
+  for (; c >= 0; --c) {
     const int64_t kk = first + c;
     const int64_t idx = (kk * g.H + h) * NP + e;
     const float s = bw.dstates[idx];
@@ -126,29 +143,63 @@ __global__ void __launch_bounds__(256) kb_state_pass(Geom g, Args a, GradArgs ga
   (void)a;
 }
 
-// acc[i][j] += sum_{k<64} A(m, k) B(k, n) with m = 4 ty + i, n = 4 tx + j.
-// A is stored [m][k] (AT false) or [k][m] (AT true); B is [k][n] (BT false) or [n][k].
-template <bool AT, bool BT>
-__device__ __forceinline__ void mac(float (&acc)[4][4], const float* A, const float* B, int ty, int tx) {
-#pragma unroll 4
-  for (int k = 0; k < 64; ++k) {
-    float av[4], bv[4];
+// acc[i][j] += sum_{k<64} A(m, k) B(k, n) with m = 4 ty + i, n = 4 tx + j, B stored
+// [k][n].  mac_nn: A stored [m][k]; mac_tn: A stored [k][m].  All shared-memory reads
+// are 16-byte vectors.
+__device__ __forceinline__ float pick(const float4& v, int q) {
+  return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+}
+
+__device__ __forceinline__ void fma_row(float (&r)[4], float a, const float4& b) {
+  r[0] = fmaf(a, b.x, r[0]);
+  r[1] = fmaf(a, b.y, r[1]);
+  r[2] = fmaf(a, b.z, r[2]);
+  r[3] = fmaf(a, b.w, r[3]);
+}
+
+__device__ __forceinline__ void mac_nn(float (&acc)[4][4], const float* A, const float* B, int ty,
+                                       int tx) {
+#pragma unroll 2
+  for (int k0 = 0; k0 < 64; k0 += 4) {
+    float4 a[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) av[i] = AT ? A[k * kLD + 4 * ty + i] : A[(4 * ty + i) * kLD + k];
+    for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(A + (4 * ty + i) * kLD + k0);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) bv[j] = BT ? B[(4 * tx + j) * kLD + k] : B[k * kLD + 4 * tx + j];
+    for (int q = 0; q < 4; ++q) {
+      const float4 b = *reinterpret_cast<const float4*>(B + (k0 + q) * kLD + 4 * tx);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      for (int i = 0; i < 4; ++i) fma_row(acc[i], pick(a[i], q), b);
+    }
   }
 }
 
+__device__ __forceinline__ void mac_tn(float (&acc)[4][4], const float* A, const float* B, int ty,
+                                       int tx) {
+#pragma unroll 4
+  for (int k = 0; k < 64; ++k) {
+    const float4 a = *reinterpret_cast<const float4*>(A + k * kLD + 4 * ty);
+    const float4 b = *reinterpret_cast<const float4*>(B + k * kLD + 4 * tx);
+    fma_row(acc[0], a.x, b);
+    fma_row(acc[1], a.y, b);
+    fma_row(acc[2], a.z, b);
+    fma_row(acc[3], a.w, b);
+  }
+}
+
+// T[r][c] = f(r, c), and its transpose T[c][r] = f(r, c), for r, c < 64 (c is the
+// contiguous index of the source, so the global reads coalesce either way)
 template <class F>
 __device__ __forceinline__ void fill(float* T, F f) {
   for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
     const int r = e >> 6, c = e & 63;
     T[r * kLD + c] = f(r, c);
+  }
+}
+template <class F>
+__device__ __forceinline__ void fill_t(float* T, F f) {
+  for (int e = threadIdx.x; e < 64 * 64; e += blockDim.x) {
+    const int r = e >> 6, c = e & 63;
+    T[c * kLD + r] = f(r, c);
   }
 }
 
@@ -233,9 +284,9 @@ __global__ void __launch_bounds__(256) kb_chunk(Geom g, Args a, GradArgs ga, Sim
     float acc[4][4] = {};
     for (int p0 = 0; p0 < P; p0 += 64) {
       fill(TA, [&](int r, int c) { return xv(r, p0 + c); });
-      fill(TB, [&](int r, int c) { return dyv(r, p0 + c); });
+      fill_t(TB, [&](int r, int c) { return dyv(r, p0 + c); });
       __syncthreads();
-      mac<false, true>(acc, TA, TB, ty, tx);  // acc = <x_s, dy_t>, s = 4ty+i, t = 4tx+j
+      mac_nn(acc, TA, TB, ty, tx);  // acc = <x_s, dy_t>, s = 4ty+i, t = 4tx+j
       __syncthreads();
     }
 #pragma unroll
@@ -252,9 +303,9 @@ __global__ void __launch_bounds__(256) kb_chunk(Geom g, Args a, GradArgs ga, Sim
     float acc[4][4] = {};
     for (int n0 = 0; n0 < N; n0 += 64) {
       fill(TA, [&](int r, int c) { return cv(r, n0 + c); });
-      fill(TB, [&](int r, int c) { return bv(r, n0 + c); });
+      fill_t(TB, [&](int r, int c) { return bv(r, n0 + c); });
       __syncthreads();
-      mac<false, true>(acc, TA, TB, ty, tx);  // acc = <C_u, B_s>, u = 4ty+i, s = 4tx+j
+      mac_nn(acc, TA, TB, ty, tx);  // acc = <C_u, B_s>, u = 4ty+i, s = 4tx+j
       __syncthreads();
     }
 #pragma unroll
@@ -272,20 +323,21 @@ __global__ void __launch_bounds__(256) kb_chunk(Geom g, Args a, GradArgs ga, Sim
     fill(TB, [&](int r, int c) { return vdl[r] * bv(r, n0 + c); });
     fill(TC, [&](int r, int c) { return cv(r, n0 + c); });
     __syncthreads();
-    float aC[4][4] = {}, aB[4][4] = {}, aC2[4][4] = {}, aB2[4][4] = {};
-    mac<false, false>(aC, W, TB, ty, tx);  // sum_s W[t][s] delta_s B_s[n]
-    mac<true, false>(aB, W, TC, ty, tx);   // sum_u W[u][s] C_u[n]
+    // the inter-chunk terms go into the same accumulators through row-scaled tiles
+    float aC[4][4] = {}, aB[4][4] = {};
+    mac_nn(aC, W, TB, ty, tx);  // sum_s W[t][s] delta_s B_s[n]
+    mac_tn(aB, W, TC, ty, tx);  // sum_u W[u][s] C_u[n]
     for (int p0 = 0; p0 < P; p0 += 64) {
       __syncthreads();
-      fill(TA, [&](int r, int c) { return dyv(r, p0 + c); });
-      fill(TD, [&](int r, int c) { return st(Hc, n0 + r, p0 + c); });
+      fill(TA, [&](int r, int c) { return vecs[r] * dyv(r, p0 + c); });
+      fill_t(TD, [&](int r, int c) { return st(Hc, n0 + r, p0 + c); });
       __syncthreads();
-      mac<false, true>(aC2, TA, TD, ty, tx);  // sum_p dy_t[p] H_c[n][p]
+      mac_nn(aC, TA, TD, ty, tx);  // + exp(cs_t) sum_p dy_t[p] H_c[n][p]
       __syncthreads();
-      fill(TA, [&](int r, int c) { return xv(r, p0 + c); });
-      fill(TD, [&](int r, int c) { return st(dE, n0 + r, p0 + c); });
+      fill(TA, [&](int r, int c) { return veq[r] * xv(r, p0 + c); });
+      fill_t(TD, [&](int r, int c) { return st(dE, n0 + r, p0 + c); });
       __syncthreads();
-      mac<false, true>(aB2, TA, TD, ty, tx);  // sum_p x_s[p] dE[n][p]
+      mac_nn(aB, TA, TD, ty, tx);  // + exp(cs_last - cs_s) sum_p x_s[p] dE[n][p]
     }
     float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -294,8 +346,8 @@ __global__ void __launch_bounds__(256) kb_chunk(Geom g, Args a, GradArgs ga, Sim
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int n = n0 + 4 * tx + j;
-        const float dc = fmaf(vecs[r], aC2[i][j], aC[i][j]);
-        const float db = vdl[r] * fmaf(veq[r], aB2[i][j], aB[i][j]);
+        const float dc = aC[i][j];
+        const float db = vdl[r] * aB[i][j];
         if (r < len && n < N) {
           const int64_t o = ((t0 + r) * G + grp) * N + n;
           atomicAdd(ga.dC + o, dc);
@@ -318,14 +370,14 @@ __global__ void __launch_bounds__(256) kb_chunk(Geom g, Args a, GradArgs ga, Sim
     fill(TA, [&](int r, int c) { return dyv(r, p0 + c); });
     fill(TC, [&](int r, int c) { return xv(r, p0 + c); });
     __syncthreads();
-    float acc[4][4] = {}, acc2[4][4] = {};
-    mac<true, false>(acc, V, TA, ty, tx);  // sum_u V[u][s] dy_u[p]
+    float acc[4][4] = {};
+    mac_tn(acc, V, TA, ty, tx);  // sum_u V[u][s] dy_u[p]
     for (int n0 = 0; n0 < N; n0 += 64) {
       __syncthreads();
-      fill(TB, [&](int r, int c) { return bv(r, n0 + c); });
+      fill(TB, [&](int r, int c) { return veq[r] * bv(r, n0 + c); });
       fill(TD, [&](int r, int c) { return st(dE, n0 + r, p0 + c); });
       __syncthreads();
-      mac<false, false>(acc2, TB, TD, ty, tx);  // sum_n B_s[n] dE[n][p]
+      mac_nn(acc, TB, TD, ty, tx);  // + exp(cs_last - cs_s) sum_n B_s[n] dE[n][p]
     }
     float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -334,7 +386,7 @@ __global__ void __launch_bounds__(256) kb_chunk(Geom g, Args a, GradArgs ga, Sim
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int p = p0 + 4 * tx + j;
-        const float gb = fmaf(veq[s], acc2[i][j], acc[i][j]);
+        const float gb = acc[i][j];
         if (s < len && p < P)
           ga.dx[((t0 + s) * H + h) * P + p] = fmaf(vdl[s], gb, Dh * TA[s * kLD + 4 * tx + j]);
         part[i] = fmaf(TC[s * kLD + 4 * tx + j], gb, part[i]);

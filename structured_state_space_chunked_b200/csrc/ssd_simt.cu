@@ -209,7 +209,24 @@ __global__ void __launch_bounds__(256) k_state_pass(Geom g, Args a, SimtWorkspac
   }
   const int64_t so = ((int64_t)d * g.H + h) * NP + e;
   float hc = a.init ? a.init[so] : 0.f;
-  for (int64_t c = 0; c < cnt; ++c) {
+  // eight chunks per round: their loads are all issued before the dependent updates
+  constexpr int kU = 8;
+  int64_t c = 0;
+  for (; c + kU <= cnt; c += kU) {
+    float s[kU], dec[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t kk = first + c + u;
+      s[u] = ws.states[(kk * g.H + h) * NP + e];
+      dec[u] = ws.cs[((int64_t)h * g.nchunks_max + kk) * g.Q + g.Q - 1];
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      ws.states[((first + c + u) * g.H + h) * NP + e] = hc;
+      hc = expf(dec[u]) * hc + s[u];
+    }
+  }
+  for (; c < cnt; ++c) {
     const int64_t kk = first + c;
     const int64_t idx = (kk * g.H + h) * NP + e;
     const float s = ws.states[idx];
