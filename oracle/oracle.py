@@ -12,6 +12,7 @@ either implicitly (``batch`` rows of ``seqlen`` tokens) or by ``cu_seqlens``
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -220,3 +221,49 @@ def oracle_backward(x, dt, A, B, C, dy, D=None, dt_bias=None, initial_states=Non
         "dA": dA_part.sum(axis=0), "dB": dB.reshape(bsz, L, G, N), "dC": dC.reshape(bsz, L, G, N),
         "dD": dD_part.sum(axis=0), "ddt_bias": db_part.sum(axis=0), "dinitial_states": dinit,
     }
+
+
+FMAP_NONE, FMAP_SILU, FMAP_RELU, FMAP_BASED, FMAP_REBASED = 0, 1, 2, 3, 4
+
+
+def oracle_feature_map(X, kind):
+    """A kernel feature map on the last axis of X, in float64 ("Transformers are
+    SSMs", paperlayer.ai summary: §7.3 feature maps, SiLU by default; App. D.4 the
+    Based map, the second-order Taylor expansion of exp, and the ReBased map x (x) x).
+    The outer products are flattened row-major."""
+    X = _f64(X)
+    if kind == FMAP_NONE:
+        return X
+    if kind == FMAP_SILU:
+        return X / (1.0 + np.exp(-X))
+    if kind == FMAP_RELU:
+        return np.maximum(X, 0.0)
+    outer = (X[..., :, None] * X[..., None, :]).reshape(*X.shape[:-1], -1)
+    if kind == FMAP_REBASED:
+        return outer
+    if kind == FMAP_BASED:
+        ones = np.ones(X.shape[:-1] + (1,))
+        return np.concatenate([ones, X, outer / math.sqrt(2.0)], axis=-1)
+    raise ValueError(f"unknown feature map {kind}")
+
+
+def oracle_forward_ext(x, dt, A, B, C, D=None, dt_bias=None, feature_map=FMAP_SILU,
+                       normalize=False, cu_seqlens=None):
+    """The scan with the feature map on B and C and, optionally, the denominator
+    normalisation of §7.3: the numerator is the scan on x with no skip term, the
+    denominator the same scan on a column of ones (X augmented with ones), and
+    y = num / den + D x.  Returns (y, final_states of the numerator)."""
+    x64 = _f64(x)
+    D64 = None if D is None else _f64(D)
+    Bf = oracle_feature_map(B, feature_map)
+    Cf = oracle_feature_map(C, feature_map)
+    if not normalize:
+        return oracle_forward(x64, dt, A, Bf, Cf, D64, dt_bias, cu_seqlens=cu_seqlens)
+    num, fin = oracle_forward(x64, dt, A, Bf, Cf, None, dt_bias, cu_seqlens=cu_seqlens)
+    den, _ = oracle_forward(np.ones(x64.shape[:-1] + (1,)), dt, A, Bf, Cf, None, dt_bias,
+                            cu_seqlens=cu_seqlens)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        y = num / den
+    if D64 is not None:
+        y = y + D64[None, None, :, None] * x64
+    return y, fin

@@ -367,3 +367,74 @@ def test_backward_head_subset_matches_full_run():
         assert np.array_equal(part["dinitial_states"][:, h], full["dinitial_states"][:, h])
         assert part["dA"][h] == full["dA"][h]
     assert np.isnan(part["dx"][:, :, 0]).all()
+
+
+# ---- feature maps and denominator normalisation ---------------------------------------
+
+def test_pointwise_feature_maps_match_library_functions():
+    from scipy.special import expit
+    X = np.random.default_rng(1).standard_normal((5, 3, 7)) * 4
+    assert np.allclose(oracle.oracle_feature_map(X, oracle.FMAP_SILU), X * expit(X), rtol=1e-14)
+    assert np.array_equal(oracle.oracle_feature_map(X, oracle.FMAP_RELU), np.clip(X, 0, None))
+    assert np.array_equal(oracle.oracle_feature_map(X, oracle.FMAP_NONE), X)
+
+
+def test_based_and_rebased_maps_are_the_kernels_they_approximate():
+    r = np.random.default_rng(2)
+    a, b = r.standard_normal(6), r.standard_normal(6)
+    dot = float(a @ b)
+    fa, fb = (oracle.oracle_feature_map(v[None], oracle.FMAP_BASED)[0] for v in (a, b))
+    assert fa.shape == (1 + 6 + 36,)
+    assert abs(fa @ fb - (1 + dot + dot * dot / 2)) < 1e-12      # Taylor of exp to 2nd order
+    ga, gb = (oracle.oracle_feature_map(v[None], oracle.FMAP_REBASED)[0] for v in (a, b))
+    assert ga.shape == (36,)
+    assert abs(ga @ gb - dot * dot) < 1e-12
+
+
+def test_normalised_scan_equals_normalised_linear_attention_when_A_is_zero():
+    """A = 0 removes the decay: y_t = sum_{s<=t} w_ts x_s / sum_{s<=t} w_ts with
+    w_ts = delta_s <phi(C_t), phi(B_s)>, written out directly (plus D x)."""
+    r = np.random.default_rng(3)
+    L, H, P, N = 9, 2, 3, 8
+    x = r.standard_normal((1, L, H, P))
+    dt = r.standard_normal((1, L, H))
+    A = np.zeros(H)
+    Bm, Cm = r.standard_normal((1, L, 1, N)), r.standard_normal((1, L, 1, N))
+    D = r.standard_normal(H)
+    bias = r.uniform(-0.5, 0.5, H)
+    for kind in (oracle.FMAP_RELU, oracle.FMAP_BASED, oracle.FMAP_REBASED):
+        y, _ = oracle.oracle_forward_ext(x, dt, A, Bm, Cm, D, bias, kind, normalize=True)
+        fB = oracle.oracle_feature_map(Bm[0, :, 0], kind)
+        fC = oracle.oracle_feature_map(Cm[0, :, 0], kind)
+        delta = np.logaddexp(0.0, dt[0] + bias)                         # [L, H]
+        assert np.isfinite(y).mean() > 0.8      # ReLU can leave a token with no weight (0 / 0)
+        for h in range(H):
+            for t in range(L):
+                w = np.array([delta[s, h] * (fC[t] @ fB[s]) for s in range(t + 1)])
+                with np.errstate(invalid="ignore"):
+                    ref = (w[:, None] * x[0, :t + 1, h]).sum(0) / w.sum() + D[h] * x[0, t, h]
+                with np.errstate(invalid="ignore"):
+                    assert np.allclose(y[0, t, h], ref, rtol=1e-11, atol=1e-12, equal_nan=True)
+
+
+def test_normalised_scan_of_a_constant_input_returns_it():
+    r = np.random.default_rng(4)
+    L, H, P, N = 40, 3, 5, 4
+    v = r.standard_normal(P)
+    x = np.broadcast_to(v, (2, L, H, P)).copy()
+    dt = r.standard_normal((2, L, H))
+    A = -np.exp(r.uniform(0, 2, H))
+    Bm, Cm = r.standard_normal((2, L, 1, N)), r.standard_normal((2, L, 1, N))
+    for kind in (oracle.FMAP_RELU, oracle.FMAP_BASED, oracle.FMAP_REBASED):
+        y, _ = oracle.oracle_forward_ext(x, dt, A, Bm, Cm, None, None, kind, normalize=True)
+        ok = np.isfinite(y)
+        assert ok.mean() > 0.9
+        assert np.allclose(y[ok], np.broadcast_to(v, y.shape)[ok], rtol=1e-9)
+
+
+def test_feature_map_without_normalisation_is_the_plain_scan_of_mapped_inputs():
+    x, dt, A, Bm, Cm, D, bias, _ = _rand(5, 2, 21, 3, 4, 3, 1)
+    y, fin = oracle.oracle_forward_ext(x, dt, A, Bm, Cm, D, bias, oracle.FMAP_SILU)
+    y2, fin2 = oracle.oracle_forward(x, dt, A, Bm / (1 + np.exp(-Bm)), Cm / (1 + np.exp(-Cm)), D,
+                                     bias)
+    assert np.array_equal(y, y2) and np.array_equal(fin, fin2)
