@@ -401,6 +401,94 @@ def run_bwd(args, w, rank, world, local, pg, hbm_peak, peak_kind):
         pg.destroy_process_group()
 
 
+def run_ext(args, w, rank, world, local, pg, hbm_peak, peak_kind):
+    """--op ext: ``ssd_forward_ext`` over the workload with the ReLU feature map on B
+    and C and the denominator normalisation (the scan of a ones column).
+
+    Compulsory bytes: B and C read and their mapped copies written; the numerator
+    scan's x, dt, mapped B and C read, y written, final states written; the
+    denominator scan's dt, mapped B and C read and its output written;
+    the division's y read and written, x and the denominator read.  L2 is flushed
+    before every timed step.
+    """
+    import torch
+
+    from structured_state_space_chunked_b200 import inputs as I
+    from structured_state_space_chunked_b200 import ssd
+
+    if w.varlen_tokens:
+        raise SystemExit("--op ext takes a batch-mode workload")
+    dev = torch.device("cuda", local)
+    inp = I.make_inputs(w, device=dev)
+    bsz, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    fmap = ssd.SSD_FMAP_RELU
+    N2 = ssd.feature_map_dim(fmap, N)
+    h = ssd.SSD(bsz, L, H, P, N, G, w.torch_dtype, device=dev)
+    y = torch.empty(bsz, L, H, P, dtype=w.torch_dtype, device=dev)
+    fin = torch.empty(bsz, H, N2, P, dtype=torch.float32, device=dev)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        h.forward_ext(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["dt_bias"],
+                      w.chunk_size, feature_map=fmap, normalize=True, y=y, final_states=fin)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if h.status() != 0:
+        raise SystemExit("device status set during warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.2)
+    barrier(pg)
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    barrier(pg)
+    t_wall1 = time.time()
+    clk.region(t_wall0, t_wall1)
+    time.sleep(0.1)
+    clocks = clk.stop()
+    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    ms = max_over_ranks(pg, ms)
+    es = 2 if w.dtype == "bf16" else 4
+    T = bsz * L
+    byts = (2 * T * G * (N + N2) * es
+            + T * H * P * es + T * H * es + 2 * T * G * N2 * es + T * H * P * es + bsz * H * N2 * P * 4
+            + T * H * es + 2 * T * G * N2 * es + T * H * 4
+            + 2 * T * H * P * es + T * H * P * es + T * H * 4)
+    achieved = byts / (ms * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": "SSD forward with ReLU feature map and denominator normalisation (ssd_forward_ext) "
+                      "Mtokens/s and % of HBM roofline",
+            "value": T * world / (ms * 1e-3) / 1e6, "unit": "Mtokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "feature_map": "relu", "normalize": True, "batch": bsz,
+                       "seqlen": L, "nheads": H, "headdim": P, "dstate": N, "ngroups": G,
+                       "parallelism": f"dp{world} (independent replicas)",
+                       "l2": "flushed before every timed step (512 MiB write, outside the events)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None,
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == "measured"
+                         else "fallback", "algorithmic_bytes_per_launch": byts,
+                         "kernel": "fmap_kernel x2 + ssd_tc_fused + den_scan_kernel + normalize_kernel"},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": 5 * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
 def run_cp(args, w, rank, world, local, pg, hbm_peak, peak_kind):
     """--op cp: the device steps one context-parallel rank adds to its own forward.
 
@@ -510,12 +598,14 @@ def main():
                     help="column width of the tensor-core kernel's work units")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--op", default="forward", choices=["forward", "step", "cp", "backward"],
+    ap.add_argument("--op", default="forward",
+                    choices=["forward", "step", "cp", "backward", "ext"],
                     help="forward: the chunked scan (default); step: one decode token per "
                          "sequence (ssd_step) with the workload's head shape; cp: the device "
                          "steps a context-parallel rank adds to its forward (log decay, "
                          "combine over --cp-ranks ranks, output correction), the workload "
-                         "being the rank's slice; backward: ssd_backward over the workload")
+                         "being the rank's slice; backward: ssd_backward over the workload; "
+                         "ext: ssd_forward_ext with the ReLU feature map and normalisation")
     ap.add_argument("--cp-ranks", type=int, default=4, help="ranks for --op cp")
     ap.add_argument("--decode-batch", type=int, default=256,
                     help="sequences per ssd_step call (--op step)")
@@ -538,6 +628,9 @@ def main():
         return
     if args.op == "backward":
         run_bwd(args, w, rank, world, local, pg, hbm_peak, peak_kind)
+        return
+    if args.op == "ext":
+        run_ext(args, w, rank, world, local, pg, hbm_peak, peak_kind)
         return
 
     if args.impl == "reference":

@@ -227,6 +227,51 @@ SSD_API int ssd_backward(ssd_handle_t h, const void* x, const void* dt, const fl
                          float* dinitial_states, ssd_stream_t stream);
 
 /*
+ * Feature maps and denominator normalisation ("Transformers are SSMs", paperlayer.ai
+ * summary: §7.3, SSD extensions taken from linear attention; the kernel
+ * approximations of §9.4.3 and App. D.4).  A feature map phi is applied to each
+ * (token, group) row of B and of C before the scan:
+ *   SSD_FMAP_SILU     phi(x) = x sigmoid(x), elementwise (the default of §7.3)
+ *   SSD_FMAP_RELU     phi(x) = max(x, 0), elementwise
+ *   SSD_FMAP_BASED    phi(x) = [1, x, (x outer x) / sqrt(2)] (second-order Taylor
+ *                     expansion of exp(<a, b>)): dstate N becomes 1 + N + N^2
+ *   SSD_FMAP_REBASED  phi(x) = x outer x (row-major flattening): N becomes N^2
+ * With normalisation, y = num / den + D x, where num is the scan's output on x and
+ * den the same scan on a column of ones (§7.3: X augmented with ones); phi should
+ * be positive so that den is (ReLU, Based and ReBased are non-negative; SiLU is not).
+ */
+enum {
+  SSD_FMAP_NONE = 0,
+  SSD_FMAP_SILU = 1,
+  SSD_FMAP_RELU = 2,
+  SSD_FMAP_BASED = 3,
+  SSD_FMAP_REBASED = 4
+};
+
+/* dstate of the scan after feature map `kind` on an input of dstate N; -1 if unknown. */
+SSD_API int ssd_feature_map_dim(int kind, int dstate);
+
+/*
+ * ssd_forward_ext: ssd_forward with a feature map on B and C and optional
+ * normalisation.  The handle's desc gives the input dstate N of B and C; the scan
+ * runs with N' = ssd_feature_map_dim(feature_map, N) (which the tensor-core path
+ * takes when N' is a multiple of 16 up to 256, else the CUDA-core path).  Arguments
+ * as for ssd_forward, except:
+ *   no initial states (the denominator's state would need one of its own);
+ *   final_states [docs, H, N', P] fp32 or NULL: the numerator's final states;
+ *   normalize 0 or 1.
+ * The mapped B and C and the denominator live in the handle's workspace.  The
+ * denominator runs as its own single-column scan (one warp per document and head)
+ * and takes N' up to 1024.  Errors as for ssd_forward; SSD_ERR_INVALID_ARG for an
+ * unknown map, SSD_ERR_UNSUPPORTED for a normalised N' over 1024.
+ */
+SSD_API int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* A,
+                            const void* B, const void* C, const float* D, const float* dt_bias,
+                            int chunk_size, const int32_t* cu_seqlens, int num_docs,
+                            int feature_map, int normalize, void* y, float* final_states,
+                            ssd_stream_t stream);
+
+/*
  * ssd_get_status: synchronises `stream`, returns the first device-side error
  * recorded since the last call (SSD_OK if none) and clears it.
  */

@@ -1,6 +1,6 @@
 // ssd_api.cu -- the C ABI declared in include/ssd.h: argument checks, path
 // selection, workspace management and launches.  All compute runs in the
-// kernels of ssd_simt.cu and ssd_tc.cu.
+// kernels of ssd_simt.cu, ssd_tc.cu, ssd_tc_wide.cu, ssd_bwd.cu and ssd_ext.cu.
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -9,6 +9,7 @@
 #include <new>
 
 #include "ssd_bwd.h"
+#include "ssd_ext.h"
 #include "ssd_internal.h"
 
 struct ssd_handle_s {
@@ -258,6 +259,98 @@ int ssd_backward(ssd_handle_t h, const void* x, const void* dt, const float* A, 
   ssd::Args a{x, dt, A, B, C, D, dt_bias, initial_states, cu_seqlens, nullptr, nullptr};
   ssd::GradArgs ga{dy, dfinal_states, dx, ddt, dA, dB, dC, dD, ddt_bias, dinitial_states};
   cudaError_t e = ssd::bwd_run(g, a, ga, h->ws, h->status, stream);
+  if (cur != h->device) cudaSetDevice(cur);
+  return cuda_rc(e);
+}
+
+int ssd_feature_map_dim(int kind, int dstate) {
+  if (dstate < 1) return -1;
+  return ssd::fmap_dim(kind, dstate);
+}
+
+int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* A, const void* B,
+                    const void* C, const float* D, const float* dt_bias, int chunk_size,
+                    const int32_t* cu_seqlens, int num_docs, int feature_map, int normalize, void* y,
+                    float* final_states, ssd_stream_t stream_) {
+  if (!h) return SSD_ERR_INVALID_ARG;
+  const ssd_desc_t& d = h->desc;
+  int rc = check_call(d, chunk_size, cu_seqlens, num_docs);
+  if (rc) return rc;
+  const int N2 = ssd::fmap_dim(feature_map, (int)d.dstate);
+  if (N2 < 1 || N2 > 65536 || (normalize != 0 && normalize != 1)) return SSD_ERR_INVALID_ARG;
+  const int64_t tokens = d.batch * d.seqlen;
+  if (tokens > 0 && (!x || !dt || !B || !C || !y)) return SSD_ERR_INVALID_ARG;
+  if (!A) return SSD_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(B, elem_bytes(d.in_dtype)) || !aligned(C, elem_bytes(d.in_dtype)) ||
+      !aligned(y, 16) || !aligned(dt, elem_bytes(d.in_dtype)) || !aligned(A, 4) || !aligned(D, 4) ||
+      !aligned(dt_bias, 4) || !aligned(final_states, 16) || !aligned(cu_seqlens, 4))
+    return SSD_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  ssd_desc_t d2 = d;
+  d2.dstate = N2;
+  Geom g;
+  make_geom(d2, chunk_size, cu_seqlens != nullptr, num_docs, &g);
+  const int path = choose_path(d2, g, h->force_path);
+  if (path < 0) return path;
+  if (path == SSD_PATH_TC && h->tc_unit_columns == 128 && !ssd::tc_wide_supported(g))
+    return SSD_ERR_UNSUPPORTED;
+  if (normalize && !ssd::den_scan_supported(N2)) return SSD_ERR_UNSUPPORTED;
+  // the denominator's geometry: one column, chunks of kDenQ tokens
+  ssd_desc_t dd = d2;
+  dd.headdim = 1;
+  Geom gd;
+  make_geom(dd, ssd::kDenQ, cu_seqlens != nullptr, num_docs, &gd);
+
+  const size_t es = elem_bytes(d.in_dtype);
+  auto al = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  const size_t b_bc = al(es * (size_t)tokens * d.ngroups * N2);
+  const size_t b_den = normalize ? al(sizeof(float) * (size_t)tokens * d.nheads) : 0;
+  const size_t b_fwd = al(workspace_for(g, path));
+  const size_t b_dws = normalize ? al(ssd::simt_workspace_bytes(gd)) : 0;
+  const size_t need = 2 * b_bc + b_den + b_fwd + b_dws;
+
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return SSD_ERR_CUDA;
+  if (need > h->ws_bytes) {
+    if (h->ws) cudaFreeAsync(h->ws, stream);
+    h->ws = nullptr;
+    h->ws_bytes = 0;
+    cudaError_t e = cudaMallocAsync(&h->ws, need, stream);
+    if (e != cudaSuccess) {
+      h->ws = nullptr;
+      if (cur != h->device) cudaSetDevice(cur);
+      return cuda_rc(e);
+    }
+    h->ws_bytes = need;
+  }
+  char* base = static_cast<char*>(h->ws);
+  void* B2 = base;
+  void* C2 = base + b_bc;
+  float* den = reinterpret_cast<float*>(base + 2 * b_bc);
+  void* fws = base + 2 * b_bc + b_den;
+  void* dws = base + 2 * b_bc + b_den + b_fwd;
+  const int bf = d.in_dtype == SSD_BF16;
+  const int64_t rows = tokens * d.ngroups;
+  cudaError_t e = ssd::fmap_apply(feature_map, rows, (int)d.dstate, N2, bf, B, B2, stream);
+  if (e == cudaSuccess) e = ssd::fmap_apply(feature_map, rows, (int)d.dstate, N2, bf, C, C2, stream);
+  // the numerator (D added after the division when normalising)
+  ssd::Args a{x, dt, A, B2, C2, normalize ? nullptr : D, dt_bias, nullptr, cu_seqlens, y, final_states};
+  if (e == cudaSuccess) {
+    if (path == SSD_PATH_TC) {
+      e = ssd::tc_forward(g, a, fws, h->status, stream, h->num_sms, h->tc_unit_columns);
+    } else {
+      ssd::SimtWorkspace ws;
+      ssd::simt_carve_workspace(g, fws, &ws);
+      e = ssd::simt_forward(g, a, ws, h->status, stream);
+    }
+  }
+  if (normalize && e == cudaSuccess) {
+    e = ssd::den_scan(gd, cu_seqlens, dws, h->status, dt, A, dt_bias, B2, C2, den, stream);
+    if (e == cudaSuccess)
+      e = ssd::normalize_apply(tokens, (int)d.nheads, (int)d.headdim, d.out_dtype == SSD_BF16, bf, y,
+                               den, x, D, stream);
+  }
   if (cur != h->device) cudaSetDevice(cur);
   return cuda_rc(e);
 }

@@ -437,4 +437,10 @@ cudaError_t simt_states(const Geom& g, const Args& a, const SimtWorkspace& ws, i
   return simt_run(g, a, ws, status, stream, false);
 }
 
+cudaError_t simt_varlen_table(const Geom& g, const int32_t* cu, const SimtWorkspace& ws, int* status,
+                              cudaStream_t stream) {
+  k_varlen_table<<<1, 1024, 0, stream>>>(g, cu, ws, status);
+  return cudaGetLastError();
+}
+
 }  // namespace ssd

@@ -33,7 +33,7 @@ ABI_SYMBOLS = (
     "ssd_validate_desc", "ssd_plan", "ssd_create", "ssd_set_option", "ssd_forward",
     "ssd_forward_host", "ssd_get_status", "ssd_destroy", "ssd_error_string", "ssd_version",
     "ssd_forward_noalloc", "ssd_step", "ssd_cp_logdecay", "ssd_cp_combine", "ssd_cp_correct",
-    "ssd_backward",
+    "ssd_backward", "ssd_feature_map_dim", "ssd_forward_ext",
 )
 
 
@@ -82,6 +82,9 @@ def lib():
         L.ssd_forward_host.argtypes = fwd
         L.ssd_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp,
                                    vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.ssd_feature_map_dim.argtypes = [i32, i32]
+        L.ssd_forward_ext.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
+                                      vp, vp, vp]
         L.ssd_get_status.argtypes = [vp, vp]
         L.ssd_forward_noalloc.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp, vp, i32,
                                           vp, vp, i32, vp, vp, vp, vp]
@@ -238,6 +241,28 @@ class SSD:
             raise SSDError(rc, "ssd_forward")
         return y, final_states
 
+    def forward_ext(self, x, dt, A, B, C, D=None, dt_bias=None, chunk_size=256,
+                    feature_map=1, normalize=False, cu_seqlens=None, num_docs=None, y=None,
+                    final_states=None, return_final_states=True, stream=None):
+        """``ssd_forward_ext``: the scan with feature map ``feature_map`` (SSD_FMAP_*)
+        on B and C and, with ``normalize``, division by the scan of a ones column.
+        ``final_states`` has the mapped dstate."""
+        ndocs, y, _ = self._prepare(x, dt, A, B, C, D, dt_bias, None, cu_seqlens, num_docs, y,
+                                    None, False, True)
+        n2 = feature_map_dim(feature_map, self.desc.dstate)
+        shape = (ndocs, self.desc.nheads, n2, self.desc.headdim)
+        if final_states is None and return_final_states:
+            final_states = torch.empty(shape, dtype=torch.float32, device=self.device)
+        self._check("final_states", final_states, shape, torch.float32)
+        rc = lib().ssd_forward_ext(self._h, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                   _ptr(dt_bias), int(chunk_size), _ptr(cu_seqlens),
+                                   int(ndocs if cu_seqlens is not None else 0), int(feature_map),
+                                   int(bool(normalize)), _ptr(y), _ptr(final_states),
+                                   _stream_ptr(stream))
+        if rc:
+            raise SSDError(rc, "ssd_forward_ext")
+        return y, final_states
+
     def backward(self, x, dt, A, B, C, dy, D=None, dt_bias=None, initial_states=None,
                  dfinal_states=None, cu_seqlens=None, num_docs=None, stream=None):
         """Enqueue ``ssd_backward``: the gradient of sum <dy, y> + <dfinal_states,
@@ -294,6 +319,17 @@ class SSD:
             self.close()
         except Exception:
             pass
+
+
+SSD_FMAP_NONE, SSD_FMAP_SILU, SSD_FMAP_RELU, SSD_FMAP_BASED, SSD_FMAP_REBASED = 0, 1, 2, 3, 4
+
+
+def feature_map_dim(kind: int, dstate: int) -> int:
+    """``ssd_feature_map_dim``: dstate of the scan after feature map ``kind``."""
+    n = int(lib().ssd_feature_map_dim(int(kind), int(dstate)))
+    if n < 1:
+        raise SSDError(-1, "ssd_feature_map_dim")
+    return n
 
 
 _cache = {}

@@ -127,3 +127,9 @@ def test_backward_refuses_a_missing_handle_without_a_gpu():
     # ssd_backward checks its handle before it touches the device
     L = ssd.lib()
     assert L.ssd_backward(None, *([None] * 9), 0, *([None] * 11)) == -1  # SSD_ERR_INVALID_ARG
+
+
+def test_feature_map_dims_without_a_gpu():
+    assert [ssd.feature_map_dim(k, 8) for k in range(5)] == [8, 8, 8, 73, 64]
+    assert ssd.lib().ssd_feature_map_dim(7, 8) == -1
+    assert ssd.lib().ssd_forward_ext(None, *([None] * 7), 64, None, 0, 1, 0, None, None, None) == -1
