@@ -129,3 +129,39 @@ def test_backward_full_size_sampled_heads(name, heads):
     # dD is sum <dy, x> over the head's tokens, for every head
     dD = (dy.double() * inp["x"].double()).sum(dim=(0, 1, 3))
     assert rel_err(got["dD"], to_np(dD)) <= SUM_TOL
+
+
+def test_backward_wide_head_dim():
+    w = I.random_small(41, "fp32", 1, 150, 2, 256, 64, 1, 64, "normal0.1")
+    inp = make(w)
+    dy, dfin = I.make_cotangents(w, 1, device="cuda")
+    got = _run(w, inp, dy, dfin)
+    ref = _oracle(inp, dy, dfin)
+    for k in PER_TOKEN:
+        assert rel_err(got[k], ref[k]) <= TOK_TOL, k
+    for k in PER_HEAD:
+        assert rel_err(got[k], ref[k]) <= SUM_TOL, k
+
+
+def test_backward_of_an_empty_sequence_passes_the_final_cotangent_through():
+    h = ssd.SSD(2, 0, 2, 16, 16, 1, torch.float32)
+    e = torch.empty(2, 0, 2, 16, device="cuda")
+    A = -torch.ones(2, device="cuda")
+    bc = torch.empty(2, 0, 1, 16, device="cuda")
+    dfin = torch.randn(2, 2, 16, 16, device="cuda")
+    g = h.backward(e, torch.empty(2, 0, 2, device="cuda"), A, bc, bc, e,
+                   dfinal_states=dfin, initial_states=torch.randn(2, 2, 16, 16, device="cuda"))
+    assert h.status() == 0
+    assert torch.equal(g["dinitial_states"], dfin)
+    assert torch.all(g["dA"] == 0) and torch.all(g["dD"] == 0)
+
+
+def test_backward_bad_cu_seqlens_sets_status():
+    w = I.random_small(4, "fp32", 1, 64, 2, 16, 16, 1, 64, varlen_tokens=64)
+    inp = make(w, cu_seqlens=np.array([0, 40, 30, 64], dtype=np.int32))
+    h = ssd.SSD(1, 64, 2, 16, 16, 1, torch.float32, max_docs=3)
+    dy = torch.randn(1, 64, 2, 16, device="cuda")
+    h.backward(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], dy, inp["D"], inp["dt_bias"],
+               cu_seqlens=inp["cu_seqlens"])
+    assert h.status() == -6
+    assert h.status() == 0

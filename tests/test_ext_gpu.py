@@ -71,3 +71,12 @@ def test_unknown_feature_map_is_refused():
     h = ssd.SSD(1, 64, 2, 64, 64, 1, torch.bfloat16)
     with pytest.raises(ssd.SSDError):
         h.forward_ext(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], feature_map=9)
+
+
+def test_forward_ext_bad_cu_seqlens_sets_status():
+    w = I.random_small(4, "bf16", 1, 0, 2, 64, 64, 1, 64, "zero", 256)
+    inp = make(w, cu_seqlens=np.array([0, 200, 100, 256], dtype=np.int32))
+    h = ssd.SSD(1, 256, 2, 64, 64, 1, torch.bfloat16, max_docs=3)
+    h.forward_ext(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"], inp["dt_bias"], 64,
+                  feature_map=ssd.SSD_FMAP_RELU, normalize=True, cu_seqlens=inp["cu_seqlens"])
+    assert h.status() == -6
