@@ -237,8 +237,11 @@ int ssd_backward(ssd_handle_t h, const void* x, const void* dt, const float* A, 
       !aligned(dinitial_states, 4) || !aligned(cu_seqlens, 4))
     return SSD_ERR_INVALID_ARG;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  ssd::Args a{x, dt, A, B, C, D, dt_bias, initial_states, cu_seqlens, nullptr, nullptr};
+  ssd::GradArgs ga{dy, dfinal_states, dx, ddt, dA, dB, dC, dD, ddt_bias, dinitial_states};
   Geom g;
-  make_geom(d, ssd::kBwdQ, cu_seqlens != nullptr, num_docs, &g);
+  make_geom(d, ssd::kBwdTcQ, cu_seqlens != nullptr, num_docs, &g);
+  if (!ssd::bwd_tc_eligible(g, a, ga)) make_geom(d, ssd::kBwdQ, cu_seqlens != nullptr, num_docs, &g);
 
   int cur = 0;
   if (cudaGetDevice(&cur) != cudaSuccess) return SSD_ERR_CUDA;
@@ -256,8 +259,6 @@ int ssd_backward(ssd_handle_t h, const void* x, const void* dt, const float* A, 
     }
     h->ws_bytes = need;
   }
-  ssd::Args a{x, dt, A, B, C, D, dt_bias, initial_states, cu_seqlens, nullptr, nullptr};
-  ssd::GradArgs ga{dy, dfinal_states, dx, ddt, dA, dB, dC, dD, ddt_bias, dinitial_states};
   cudaError_t e = ssd::bwd_run(g, a, ga, h->ws, h->status, stream);
   if (cur != h->device) cudaSetDevice(cur);
   return cuda_rc(e);

@@ -38,11 +38,6 @@ namespace {
 constexpr int kLD = 68;            // row stride of the 64 x 64 shared tiles (16-byte rows)
 constexpr int kTileF = 64 * kLD;   // floats per tile
 
-struct BwdWs {
-  float* dstates;  // [nchunks, H, N, P]: per-chunk sum, then the cotangent at the chunk's end
-  float* final;    // [ndocs, H, N, P]: the forward's final states
-};
-
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 __global__ void kb_zero(float* p, int64_t n) {
@@ -450,7 +445,8 @@ size_t bwd_workspace_bytes(const Geom& g) {
 
 cudaError_t bwd_run(const Geom& g, const Args& a_in, const GradArgs& ga, void* base, int* status,
                     cudaStream_t stream) {
-  if (g.Q != kBwdQ) return cudaErrorInvalidValue;
+  const bool tc = bwd_tc_eligible(g, a_in, ga);
+  if (g.Q != (tc ? kBwdTcQ : kBwdQ)) return cudaErrorInvalidValue;
   const size_t NP = (size_t)g.N * g.P;
   SimtWorkspace ws;
   simt_carve_workspace(g, base, &ws);
@@ -484,6 +480,7 @@ cudaError_t bwd_run(const Geom& g, const Args& a_in, const GradArgs& ga, void* b
     kb_state_pass<<<dim3(g.ndocs, g.H, (unsigned)((NP + 255) / 256)), 256, 0, stream>>>(g, a, ga, ws,
                                                                                       bw);
   }
+  if (tc && g.nchunks_max > 0 && g.H > 0) return bwd_chunk_tc(g, a, ga, ws, bw, status, stream);
   if (g.nchunks_max > 0 && g.H > 0) {
     const size_t smem = kb_chunk_smem();
     e = cudaFuncSetAttribute(kb_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

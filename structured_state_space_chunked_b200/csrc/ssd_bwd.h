@@ -25,7 +25,22 @@ struct GradArgs {
   float* dinit;          // [ndocs, H, N, P] or null
 };
 
-// g.Q must be kBwdQ.
+// Chunk length of the tensor-core backward (bf16 inputs and outputs, P = 64, N = 64 or
+// 128, 16-byte aligned x, dy, B and C); ssd_backward takes it when bwd_tc_eligible.
+constexpr int kBwdTcQ = 128;
+bool bwd_tc_eligible(const Geom& g, const Args& a, const GradArgs& ga);
+
+// Backward workspace beyond the CUDA-core forward's.
+struct BwdWs {
+  float* dstates;  // [nchunks, H, N, P]: per-chunk sum, then the cotangent at the chunk's end
+  float* final;    // [ndocs, H, N, P]: the forward's final states
+};
+
+// every per-token gradient of each (chunk, head) on the tensor cores (g.Q == kBwdTcQ)
+cudaError_t bwd_chunk_tc(const Geom& g, const Args& a, const GradArgs& ga, const SimtWorkspace& ws,
+                         const BwdWs& bw, int* status, cudaStream_t stream);
+
+// g.Q must be kBwdQ, or kBwdTcQ when bwd_tc_eligible.
 size_t bwd_workspace_bytes(const Geom& g);
 cudaError_t bwd_run(const Geom& g, const Args& a, const GradArgs& ga, void* workspace, int* status,
                     cudaStream_t stream);
