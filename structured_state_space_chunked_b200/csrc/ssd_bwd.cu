@@ -49,8 +49,8 @@ __global__ void kb_zero(float* p, int64_t n) {
 // dS_c[n][p] = sum_l exp(cs_l) C[l][n] dy[l][p] over the tokens of chunk c
 __global__ void __launch_bounds__(256) kb_chunk_dstate(Geom g, Args a, GradArgs ga, SimtWorkspace ws,
                                                        BwdWs bw) {
-  __shared__ float Cs[32][65];
-  __shared__ float Ys[32][65];
+  __shared__ __align__(16) float Cs[32][68];  // rows padded to 16-byte multiples
+  __shared__ __align__(16) float Ys[32][68];
   __shared__ float w[32];
   const int64_t k = blockIdx.x;
   const int h = blockIdx.y;
@@ -80,10 +80,13 @@ __global__ void __launch_bounds__(256) kb_chunk_dstate(Geom g, Args a, GradArgs 
     __syncthreads();
 #pragma unroll 4
     for (int r = 0; r < 32; ++r) {
+      const float4 av = *reinterpret_cast<const float4*>(&Cs[r][tn * 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&Ys[r][tp * 4]);
+      const float a4[4] = {av.x, av.y, av.z, av.w}, b4[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(Cs[r][tn * 4 + i], Ys[r][tp * 4 + j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
     }
     __syncthreads();
   }

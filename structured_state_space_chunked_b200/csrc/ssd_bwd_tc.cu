@@ -2,8 +2,9 @@
 //
 // The same chunk-level derivative as ssd_bwd.cu's kb_chunk ("Transformers are SSMs",
 // paperlayer.ai summary: the block decomposition of §6, differentiated), for bf16
-// inputs with P = 64 and N = 64 or 128, on 128-token chunks.  One CTA of 128 threads
-// per (chunk, head); thread r owns row r of every 128-row accumulator.  Every matrix
+// inputs with P = 64 and N = 64 or 128, on 128-token chunks.  One CTA of 256 threads
+// per (chunk, head); threads r and r + 128 own row r of every 128-row accumulator, each
+// half of its columns.  Every matrix
 // is staged once in shared memory as bf16 128-byte-swizzled panels and read by the
 // MMAs either K-major or MN-major:
 //
@@ -58,6 +59,12 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int* sta
   return true;
 }
 
+// four fp32 additions into 16-byte-aligned global memory, one reduction instruction
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 // v ~ hi + lo in bf16: two packed pairs
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
   hi = pack_bf16(a, b);
@@ -75,7 +82,7 @@ __device__ __forceinline__ void ld_bf16x8(uint32_t base, uint32_t panel_bytes, i
   }
 }
 
-__global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUtensorMap tm_x,
+__global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CUtensorMap tm_x,
                                                    const __grid_constant__ CUtensorMap tm_dy,
                                                    const __grid_constant__ CUtensorMap tm_b,
                                                    const __grid_constant__ CUtensorMap tm_c,
@@ -84,9 +91,11 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
   __shared__ uint64_t bars[2];
   __shared__ uint32_t tslot;
   __shared__ float vcs[kQ], vdl[kQ], vecs[kQ], veq[kQ], vdcs[kQ], vxg[kQ];
-  __shared__ float red[4];
+  __shared__ float red[8];
+  __shared__ float vpart[2][kQ];
   const Geom& g = kp.g;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // 256 threads: thread (r, half) owns row r of the accumulators and half of the columns
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, r = tid & (kQ - 1), half = tid >> 7;
   const int64_t k = blockIdx.x;
   const int h = blockIdx.y;
   ChunkInfo ci;
@@ -117,7 +126,7 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
   }
   const int64_t cso = ((int64_t)h * g.nchunks_max + k) * g.Q;
   const float cs_last = kp.ws.cs[cso + g.Q - 1];
-  {
+  if (tid < kQ) {
     const float c = kp.ws.cs[cso + tid];
     vcs[tid] = c;
     vdl[tid] = kp.ws.delta[cso + tid];
@@ -129,27 +138,40 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
   // the entering state and the end-of-chunk cotangent as bf16 operands (rows n)
   const float* Hc = kp.ws.states + (k * H + h) * NP;
   const float* dE = kp.bw.dstates + (k * H + h) * NP;
-  for (int i = tid; i < N * 8; i += 128) {
-    const int n = i >> 3, c = i & 7;
-    const float4* ph = reinterpret_cast<const float4*>(Hc + (int64_t)n * P + 8 * c);
-    const float4* pe = reinterpret_cast<const float4*>(dE + (int64_t)n * P + 8 * c);
-    const float4 h0 = ph[0], h1 = ph[1], e0 = pe[0], e1 = pe[1];
-    st_shared_v4(s_hc + swz((uint32_t)n, (uint32_t)c), pack_bf16(h0.x, h0.y), pack_bf16(h0.z, h0.w),
-                 pack_bf16(h1.x, h1.y), pack_bf16(h1.z, h1.w));
-    uint32_t eh[4], el[4];
-    split2(e0.x, e0.y, eh[0], el[0]);
-    split2(e0.z, e0.w, eh[1], el[1]);
-    split2(e1.x, e1.y, eh[2], el[2]);
-    split2(e1.z, e1.w, eh[3], el[3]);
-    st_shared_v4(s_de + swz((uint32_t)n, (uint32_t)c), eh[0], eh[1], eh[2], eh[3]);
-    st_shared_v4(s_del + swz((uint32_t)n, (uint32_t)c), el[0], el[1], el[2], el[3]);
+  // two rows of 8 columns per thread per round, all loads issued before the stores
+  for (int i0 = 0; i0 < N * 8; i0 += 2 * 256) {
+    float4 hv[2][2], ev[2][2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * 256 + tid, n = i >> 3, c = i & 7;
+      const float4* ph = reinterpret_cast<const float4*>(Hc + (int64_t)n * P + 8 * c);
+      const float4* pe = reinterpret_cast<const float4*>(dE + (int64_t)n * P + 8 * c);
+      hv[u][0] = __ldg(ph);
+      hv[u][1] = __ldg(ph + 1);
+      ev[u][0] = __ldg(pe);
+      ev[u][1] = __ldg(pe + 1);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * 256 + tid, n = i >> 3, c = i & 7;
+      const float4 h0 = hv[u][0], h1 = hv[u][1], e0 = ev[u][0], e1 = ev[u][1];
+      st_shared_v4(s_hc + swz((uint32_t)n, (uint32_t)c), pack_bf16(h0.x, h0.y), pack_bf16(h0.z, h0.w),
+                   pack_bf16(h1.x, h1.y), pack_bf16(h1.z, h1.w));
+      uint32_t eh[4], el[4];
+      split2(e0.x, e0.y, eh[0], el[0]);
+      split2(e0.z, e0.w, eh[1], el[1]);
+      split2(e1.x, e1.y, eh[2], el[2]);
+      split2(e1.z, e1.w, eh[3], el[3]);
+      st_shared_v4(s_de + swz((uint32_t)n, (uint32_t)c), eh[0], eh[1], eh[2], eh[3]);
+      st_shared_v4(s_del + swz((uint32_t)n, (uint32_t)c), el[0], el[1], el[2], el[3]);
+    }
   }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tslot;
-  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   bool ok = true;
   uint32_t mma_phase = 0;
 
@@ -185,10 +207,9 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
   // E1: W' rows (hi and lo), the dD diagonal
   float dDp = 0.f;
   {
-    const int r = tid;
     const bool row = r < len;
     const float csr = vcs[r];
-    for (int c0 = 0; c0 < 128; c0 += 32) {
+    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
       float s1[32];
       tc_ld32(trow + c0, s1);
       tc_wait_ld();
@@ -237,9 +258,8 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
   tc_fence_after();
   // E2: dC (atomics over the group's heads) and <C_t, dC_t>
   if (ok) {
-    const int r = tid;
     float part = 0.f;
-    for (int c0 = 0; c0 < N; c0 += 32) {
+    for (int c0 = half * (N / 2); c0 < (half + 1) * (N / 2); c0 += 32) {
       float a[32], b[32];
       tc_ld32(trow + c0, a);
       tc_ld32(trow + N + c0, b);
@@ -248,23 +268,25 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
         float* dst = kp.ga.dC + ((t0 + r) * G + grp) * (int64_t)N + c0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          float cv[8];
+          float cv[8], dc[8];
           ld_bf16x8(s_c, kPanel, r, (c0 >> 3) + q, cv);
 #pragma unroll
           for (int z = 0; z < 8; ++z) {
             const int j = 8 * q + z;
-            const float dc = fmaf(vecs[r], b[j], a[j]);
-            atomicAdd(dst + j, dc);
-            part = fmaf(cv[z], dc, part);
+            dc[z] = fmaf(vecs[r], b[j], a[j]);
+            part = fmaf(cv[z], dc[z], part);
           }
+          red_add4(dst + 8 * q, dc[0], dc[1], dc[2], dc[3]);
+          red_add4(dst + 8 * q + 4, dc[4], dc[5], dc[6], dc[7]);
         }
       }
     }
-    vdcs[r] = part;
+    vpart[half][r] = part;
   }
   tc_fence_before();
   ok = __syncthreads_and(ok);
   tc_fence_after();
+  if (tid < kQ) vdcs[tid] = vpart[0][tid] + vpart[1][tid];
 
   // phase C: dB = W'^T C (cols 0..N-1) and X dE^T (cols N..2N-1)
   if (ok && tid == 0) {
@@ -284,9 +306,8 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
   tc_fence_after();
   // E3: dB
   if (ok) {
-    const int r = tid;
     const float f2 = vdl[r] * veq[r];
-    for (int c0 = 0; c0 < N; c0 += 32) {
+    for (int c0 = half * (N / 2); c0 < (half + 1) * (N / 2); c0 += 32) {
       float a[32], b[32];
       tc_ld32(trow + c0, a);
       tc_ld32(trow + N + c0, b);
@@ -294,7 +315,9 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
       if (r < len) {
         float* dst = kp.ga.dB + ((t0 + r) * G + grp) * (int64_t)N + c0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) atomicAdd(dst + j, fmaf(f2, b[j], a[j]));
+        for (int j = 0; j < 32; j += 4)
+          red_add4(dst + j, fmaf(f2, b[j], a[j]), fmaf(f2, b[j + 1], a[j + 1]), fmaf(f2, b[j + 2], a[j + 2]),
+                   fmaf(f2, b[j + 3], a[j + 3]));
       }
     }
   }
@@ -304,10 +327,9 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
 
   // EV: V rows (hi and lo) from S2, into the space W' no longer needs
   if (ok) {
-    const int r = tid;
     const bool row = r < len;
     const float csr = vcs[r];
-    for (int c0 = 0; c0 < 128; c0 += 32) {
+    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
       float s2[32];
       tc_ld32(trow + 256 + c0, s2);
       tc_wait_ld();
@@ -357,10 +379,9 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
   tc_fence_after();
   // E4: dx and <x, gB>
   if (ok) {
-    const int r = tid;
     const float Dh = kp.a.D ? kp.a.D[h] : 0.f;
     float part = 0.f;
-    for (int c0 = 0; c0 < 64; c0 += 32) {
+    for (int c0 = half * 32; c0 < half * 32 + 32; c0 += 32) {
       float a[32], b[32];
       tc_ld32(trow + c0, a);
       tc_ld32(trow + 64 + c0, b);
@@ -384,11 +405,12 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
         }
       }
     }
-    vxg[r] = part;
+    vpart[half][r] = part;
   }
   tc_fence_before();
   ok = __syncthreads_and(ok);
   tc_fence_after();
+  if (tid < kQ) vxg[tid] = vpart[0][tid] + vpart[1][tid];
 
   // E5: <dE, S_last>, dcs and its reverse cumsum, ddt, the per-head sums
   if (ok) {
@@ -396,13 +418,26 @@ __global__ void __launch_bounds__(128) kb_chunk_tc(const __grid_constant__ CUten
     const int64_t cnt = doc_chunks(g, kp.ws, ci.doc, &first);
     const float* Hend = (k == first + cnt - 1) ? kp.bw.final + ((int64_t)ci.doc * H + h) * NP
                                                : kp.ws.states + ((k + 1) * H + h) * NP;
+    // 16-byte loads, eight in flight per thread
     float sp = 0.f;
-    for (int64_t e = tid; e < NP; e += 128) sp = fmaf(dE[e], Hend[e], sp);
+    const float4* d4 = reinterpret_cast<const float4*>(dE);
+    const float4* h4 = reinterpret_cast<const float4*>(Hend);
+    for (int64_t e0 = tid; e0 < NP / 4; e0 += 4 * 256) {
+      float4 dv[4], hv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        dv[u] = __ldg(d4 + e0 + u * 256);
+        hv[u] = __ldg(h4 + e0 + u * 256);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        sp += dv[u].x * hv[u].x + dv[u].y * hv[u].y + dv[u].z * hv[u].z + dv[u].w * hv[u].w;
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
     if (lane == 0) red[warp] = sp;
     __syncthreads();
-    const float scal = red[0] + red[1] + red[2] + red[3];
+    const float scal = red[0] + red[1] + red[2] + red[3] + red[4] + red[5] + red[6] + red[7];
     if (tid == 0) {
       float run = 0.f;
       for (int l = len - 1; l >= 0; --l) {
@@ -453,7 +488,7 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 bool bwd_tc_eligible(const Geom& g, const Args& a, const GradArgs& ga) {
   return g.in_bf16 && g.out_bf16 && g.P == 64 && (g.N == 64 || g.N == 128) && aligned16(a.x) &&
          aligned16(a.B) && aligned16(a.C) && aligned16(ga.dy) && aligned16(ga.dx) &&
-         g.tokens <= 0x7fffffffLL;
+         aligned16(ga.dB) && aligned16(ga.dC) && g.tokens <= 0x7fffffffLL;
 }
 
 cudaError_t bwd_chunk_tc(const Geom& g, const Args& a, const GradArgs& ga, const SimtWorkspace& ws,
@@ -480,7 +515,7 @@ cudaError_t bwd_chunk_tc(const Geom& g, const Args& a, const GradArgs& ga, const
   const size_t smem = kb_chunk_tc_smem(g.N);
   cudaError_t e = cudaFuncSetAttribute(kb_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kb_chunk_tc<<<dim3((unsigned)g.nchunks_max, g.H), 128, smem, stream>>>(tm_x, tm_dy, tm_b, tm_c, kp);
+  kb_chunk_tc<<<dim3((unsigned)g.nchunks_max, g.H), 256, smem, stream>>>(tm_x, tm_dy, tm_b, tm_c, kp);
   return cudaGetLastError();
 }
 

@@ -144,8 +144,8 @@ __global__ void k_cumsum(Geom g, Args a, SimtWorkspace ws) {
 // ---- K2: chunk states S_c[n,p] = sum_l B[l,n] w_l x[l,p] ---------------------------
 constexpr int kTS = 64;  // n and p tile of chunk_state
 __global__ void __launch_bounds__(256) k_chunk_state(Geom g, Args a, SimtWorkspace ws) {
-  __shared__ float Bs[32][kTS + 1];
-  __shared__ float Xs[32][kTS + 1];
+  __shared__ __align__(16) float Bs[32][68];  // rows padded to 16-byte multiples
+  __shared__ __align__(16) float Xs[32][68];
   __shared__ float w[32];
   const int64_t k = blockIdx.x;
   const int h = blockIdx.y;
@@ -175,10 +175,13 @@ __global__ void __launch_bounds__(256) k_chunk_state(Geom g, Args a, SimtWorkspa
     __syncthreads();
 #pragma unroll 4
     for (int r = 0; r < 32; ++r) {
+      const float4 av = *reinterpret_cast<const float4*>(&Bs[r][tn * 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&Xs[r][tp * 4]);
+      const float a4[4] = {av.x, av.y, av.z, av.w}, b4[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] += Bs[r][tn * 4 + i] * Xs[r][tp * 4 + j];
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
     }
     __syncthreads();
   }
