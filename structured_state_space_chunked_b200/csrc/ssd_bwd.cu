@@ -473,11 +473,25 @@ cudaError_t bwd_run(const Geom& g, const Args& a_in, const GradArgs& ga, void* b
   zero(ga.dA, g.H);
   zero(ga.dD, g.H);
   zero(ga.ddt_bias, g.H);
-  cudaError_t e = simt_states(g, a, ws, status, stream);
+  // the chunk-state products on the tensor cores when the chunk kernel is there and N = 128
+  const bool tc_states = tc && g.N == 128;
+  cudaError_t e;
+  if (tc_states) {
+    e = simt_cumsum(g, a, ws, status, stream);
+    if (e == cudaSuccess && g.nchunks_max > 0 && g.H > 0) e = bwd_states_tc(g, a, ga, ws, bw, 0, status, stream);
+    if (e == cudaSuccess) e = simt_state_pass(g, a, ws, status, stream);
+  } else {
+    e = simt_states(g, a, ws, status, stream);
+  }
   if (e != cudaSuccess) return e;
   if (g.nchunks_max > 0 && g.H > 0) {
-    const int tiles = ((g.N + 63) / 64) * ((g.P + 63) / 64);
-    kb_chunk_dstate<<<dim3((unsigned)g.nchunks_max, g.H, tiles), 256, 0, stream>>>(g, a, ga, ws, bw);
+    if (tc_states) {
+      e = bwd_states_tc(g, a, ga, ws, bw, 1, status, stream);
+      if (e != cudaSuccess) return e;
+    } else {
+      const int tiles = ((g.N + 63) / 64) * ((g.P + 63) / 64);
+      kb_chunk_dstate<<<dim3((unsigned)g.nchunks_max, g.H, tiles), 256, 0, stream>>>(g, a, ga, ws, bw);
+    }
   }
   if (g.ndocs > 0 && g.H > 0) {
     kb_state_pass<<<dim3(g.ndocs, g.H, (unsigned)((NP + 255) / 256)), 256, 0, stream>>>(g, a, ga, ws,

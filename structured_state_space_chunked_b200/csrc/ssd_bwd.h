@@ -9,6 +9,13 @@ namespace ssd {
 // entering every chunk in ws.states, and a.final_states when given (y untouched).
 cudaError_t simt_states(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
                         cudaStream_t stream);
+// the same in two parts around a chunk-state product of the caller's: the chunk table
+// and the cumsum (ws.cs, ws.delta); then, once ws.states holds each chunk's own state,
+// the state pass
+cudaError_t simt_cumsum(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
+                        cudaStream_t stream);
+cudaError_t simt_state_pass(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
+                            cudaStream_t stream);
 
 constexpr int kBwdQ = 64;  // chunk length of the backward kernels
 
@@ -35,6 +42,12 @@ struct BwdWs {
   float* dstates;  // [nchunks, H, N, P]: per-chunk sum, then the cotangent at the chunk's end
   float* final;    // [ndocs, H, N, P]: the forward's final states
 };
+
+// per (chunk, head) on the tensor cores (g.Q == kBwdTcQ, g.N == 128): mode 0 writes the
+// chunk's own state sum_t B_t^T (exp(cs_last - cs_t) delta_t x_t) into ws.states, mode 1
+// the cotangent sum sum_t C_t^T (exp(cs_t) dy_t) into bw.dstates
+cudaError_t bwd_states_tc(const Geom& g, const Args& a, const GradArgs& ga, const SimtWorkspace& ws,
+                          const BwdWs& bw, int mode, int* status, cudaStream_t stream);
 
 // every per-token gradient of each (chunk, head) on the tensor cores (g.Q == kBwdTcQ)
 cudaError_t bwd_chunk_tc(const Geom& g, const Args& a, const GradArgs& ga, const SimtWorkspace& ws,

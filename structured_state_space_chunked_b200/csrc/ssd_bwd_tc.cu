@@ -477,6 +477,101 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   }
 }
 
+// Chunk-state products on the tensor cores (N = 128, P = 64): D[n][p] = sum_t M[t][n] w_t V[t][p]
+// with (M, V, w) = (B, x, exp(cs_last - cs_t) delta_t) for the forward's chunk states and
+// (C, dy, exp(cs_t)) for the cotangent sums.  The weighted rows w_t V[t] enter as hi + lo
+// bf16 pairs (about 16 bits), M as stored (bf16).  One CTA of 128 threads per (chunk,
+// head); thread r scales token row r, then owns state row r of the accumulator.
+__global__ void __launch_bounds__(128) kb_states_tc(const __grid_constant__ CUtensorMap tm_m,
+                                                    const __grid_constant__ CUtensorMap tm_v,
+                                                    const __grid_constant__ TcParams kp, int mode) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ uint64_t bars[2];
+  __shared__ uint32_t tslot;
+  const Geom& g = kp.g;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t k = blockIdx.x;
+  const int h = blockIdx.y;
+  ChunkInfo ci;
+  if (!chunk_info(g, kp.a.cu, kp.ws, k, &ci)) return;
+  const int P = g.P, H = g.H, G = g.G, grp = h / (H / G), len = ci.len;
+  const int64_t NP = (int64_t)g.N * P, t0 = ci.start;
+  const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t s_m = sbase, s_v = s_m + 2 * kPanel, s_hi = s_v + kPanel, s_lo = s_hi + kPanel;
+  const uint32_t bar_load = su32(&bars[0]), bar_mma = su32(&bars[1]);
+  if (tid == 0) {
+    mbar_init(bar_load, 1);
+    mbar_init(bar_mma, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&tslot)),
+                 "r"(64)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tslot;
+  if (tid == 0) {
+    mbar_expect_tx(bar_load, 3 * kPanel);
+    tma_3d(s_m, &tm_m, bar_load, 0, grp, (int)t0);
+    tma_3d(s_m + kPanel, &tm_m, bar_load, 64, grp, (int)t0);
+    tma_2d(s_v, &tm_v, bar_load, h * P, (int)t0);
+  }
+  const int64_t cso = ((int64_t)h * g.nchunks_max + k) * g.Q;
+  float w = 0.f;
+  if (tid < len) {
+    const float c = kp.ws.cs[cso + tid];
+    w = mode == 0 ? expf(kp.ws.cs[cso + g.Q - 1] - c) * kp.ws.delta[cso + tid] : expf(c);
+  }
+  bool ok = wait_bar(bar_load, 0, kp.status);
+  // the weighted row of token tid, split into hi and lo
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float v[8];
+    ld_bf16x8(s_v, kPanel, tid, c, v);
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) split2(w * v[2 * m], w * v[2 * m + 1], hi[m], lo[m]);
+    const uint32_t off = swz((uint32_t)tid, (uint32_t)c);
+    st_shared_v4(s_hi + off, hi[0], hi[1], hi[2], hi[3]);
+    st_shared_v4(s_lo + off, lo[0], lo[1], lo[2], lo[3]);
+  }
+  fence_async_smem();
+  tc_fence_before();
+  ok = __syncthreads_and(ok);
+  tc_fence_after();
+  if (ok && tid == 0) {
+    const uint32_t id = idesc(128, 64, 1, 1);
+    for (int kk = 0; kk < 16; ++kk)
+      tc_mma(tmem, sdesc(s_m + (kk & 7) * 2048, kPanel, 1024),
+             sdesc(((kk & 8) ? s_lo : s_hi) + (kk & 7) * 2048, kPanel, 1024), id, kk > 0);
+    tc_commit(bar_mma);
+  }
+  if (ok) ok = wait_bar(bar_mma, 0, kp.status);
+  tc_fence_after();
+  if (ok) {
+    float* out = (mode == 0 ? kp.ws.states : kp.bw.dstates) + (k * H + h) * NP + (int64_t)tid * P;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+      float a[32];
+      tc_ld32(trow + c0, a);
+      tc_wait_ld();
+      float4* o4 = reinterpret_cast<float4*>(out + c0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) o4[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64) : "memory");
+  }
+}
+
 size_t kb_chunk_tc_smem(int N) {
   return 1024 + (size_t)kPanel * (2 + 2 * (N / 64) + 4) + (size_t)3 * N * 128;
 }
@@ -516,6 +611,36 @@ cudaError_t bwd_chunk_tc(const Geom& g, const Args& a, const GradArgs& ga, const
   cudaError_t e = cudaFuncSetAttribute(kb_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kb_chunk_tc<<<dim3((unsigned)g.nchunks_max, g.H), 256, smem, stream>>>(tm_x, tm_dy, tm_b, tm_c, kp);
+  return cudaGetLastError();
+}
+
+}  // namespace ssd
+
+namespace ssd {
+
+cudaError_t bwd_states_tc(const Geom& g, const Args& a, const GradArgs& ga, const SimtWorkspace& ws,
+                          const BwdWs& bw, int mode, int* status, cudaStream_t stream) {
+  if (g.Q != kQ || g.N != 128 || g.P != 64) return cudaErrorInvalidValue;
+  CUtensorMap tm_m, tm_v;
+  const cuuint64_t T = (cuuint64_t)g.tokens;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)g.N, (cuuint64_t)g.G, T};
+    const cuuint64_t str[2] = {(cuuint64_t)g.N * 2, (cuuint64_t)g.G * g.N * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kQ};
+    if (!tc::encode_bf16_sw128(&tm_m, mode == 0 ? a.B : a.C, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t row = (cuuint64_t)g.H * g.P;
+    const cuuint64_t dims[2] = {row, T};
+    const cuuint64_t str[1] = {row * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kQ};
+    if (!tc::encode_bf16_sw128(&tm_v, mode == 0 ? a.x : ga.dy, 2, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  TcParams kp{g, a, ga, ws, bw, status};
+  const size_t smem = 1024 + 5 * (size_t)kPanel;
+  cudaError_t e = cudaFuncSetAttribute(kb_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kb_states_tc<<<dim3((unsigned)g.nchunks_max, g.H), 128, smem, stream>>>(tm_m, tm_v, kp, mode);
   return cudaGetLastError();
 }
 

@@ -401,22 +401,29 @@ int simt_kernels(const Geom& g) {
   return n;
 }
 
+// stage = 0: everything; 1: up to the cumsum (the caller fills the chunk states);
+// 2: the state pass only
 cudaError_t simt_run(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
-                     cudaStream_t stream, bool outputs) {
+                     cudaStream_t stream, bool outputs, int stage = 0) {
   if (g.Q < 1 || g.Q > kMaxQ) return cudaErrorInvalidValue;
-  if (g.varlen) {
-    k_varlen_table<<<1, 1024, 0, stream>>>(g, a.cu, ws, status);
-  }
-  if (g.nchunks_max > 0 && g.H > 0) {
-    const int qthreads = ((g.Q + 31) / 32) * 32;
-    k_cumsum<<<dim3((unsigned)g.nchunks_max, g.H), qthreads, 0, stream>>>(g, a, ws);
-    const int tiles_s = ((g.N + kTS - 1) / kTS) * ((g.P + kTS - 1) / kTS);
-    k_chunk_state<<<dim3((unsigned)g.nchunks_max, g.H, tiles_s), 256, 0, stream>>>(g, a, ws);
+  if (stage != 2) {
+    if (g.varlen) {
+      k_varlen_table<<<1, 1024, 0, stream>>>(g, a.cu, ws, status);
+    }
+    if (g.nchunks_max > 0 && g.H > 0) {
+      const int qthreads = ((g.Q + 31) / 32) * 32;
+      k_cumsum<<<dim3((unsigned)g.nchunks_max, g.H), qthreads, 0, stream>>>(g, a, ws);
+      if (stage == 1) return cudaGetLastError();
+      const int tiles_s = ((g.N + kTS - 1) / kTS) * ((g.P + kTS - 1) / kTS);
+      k_chunk_state<<<dim3((unsigned)g.nchunks_max, g.H, tiles_s), 256, 0, stream>>>(g, a, ws);
+    }
+    if (stage == 1) return cudaGetLastError();
   }
   const int64_t NP = (int64_t)g.N * g.P;
   if (g.ndocs > 0) {
     k_state_pass<<<dim3(g.ndocs, g.H, (unsigned)((NP + 255) / 256)), 256, 0, stream>>>(g, a, ws);
   }
+  if (stage == 2) return cudaGetLastError();
   if (outputs && g.nchunks_max > 0) {
     const size_t smem =
         sizeof(float) * ((size_t)kSL * (g.N + 1) + 32 * (g.N + 1) + 32 * kSP + kSL * 33 + 32 * kSP +
@@ -438,6 +445,16 @@ cudaError_t simt_forward(const Geom& g, const Args& a, const SimtWorkspace& ws, 
 cudaError_t simt_states(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
                         cudaStream_t stream) {
   return simt_run(g, a, ws, status, stream, false);
+}
+
+cudaError_t simt_cumsum(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
+                        cudaStream_t stream) {
+  return simt_run(g, a, ws, status, stream, false, 1);
+}
+
+cudaError_t simt_state_pass(const Geom& g, const Args& a, const SimtWorkspace& ws, int* status,
+                            cudaStream_t stream) {
+  return simt_run(g, a, ws, status, stream, false, 2);
 }
 
 cudaError_t simt_varlen_table(const Geom& g, const int32_t* cu, const SimtWorkspace& ws, int* status,
