@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ uint64_t bars[2];
   __shared__ uint32_t tslot;
-  __shared__ float vcs[kQ], vdl[kQ], vecs[kQ], veq[kQ], vdcs[kQ], vxg[kQ];
+  __shared__ float vcs2[kQ], vdl[kQ], vecs[kQ], veq[kQ], vdcs[kQ], vxg[kQ];
   __shared__ float red[8];
   __shared__ float vpart[2][kQ];
   const Geom& g = kp.g;
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   const float cs_last = kp.ws.cs[cso + g.Q - 1];
   if (tid < kQ) {
     const float c = kp.ws.cs[cso + tid];
-    vcs[tid] = c;
+    vcs2[tid] = c * 1.4426950408889634f;  // log2 units for the in-chunk decay factors
     vdl[tid] = kp.ws.delta[cso + tid];
     vecs[tid] = expf(c);
     veq[tid] = expf(cs_last - c);
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   float dDp = 0.f;
   {
     const bool row = r < len;
-    const float csr = vcs[r];
+    const float csr2 = vcs2[r];
     for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
       float s1[32];
       tc_ld32(trow + c0, s1);
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
           for (int z = 0; z < 2; ++z) {
             const int j = 8 * q + 2 * m + z, s = c0 + j;
             const bool in = row && s <= r;
-            a2[z] = in ? expf(csr - vcs[s]) * vdl[s] * s1[j] : 0.f;
+            a2[z] = in ? ex2(csr2 - vcs2[s]) * vdl[s] * s1[j] : 0.f;
             if (s == r && row) dDp = s1[j];
           }
           split2(a2[0], a2[1], wh[m], wl[m]);
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   // EV: V rows (hi and lo) from S2, into the space W' no longer needs
   if (ok) {
     const bool row = r < len;
-    const float csr = vcs[r];
+    const float csr2 = vcs2[r];
     for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
       float s2[32];
       tc_ld32(trow + 256 + c0, s2);
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
 #pragma unroll
           for (int z = 0; z < 2; ++z) {
             const int j = 8 * q + 2 * m + z, s = c0 + j;
-            b2[z] = (row && s <= r) ? expf(csr - vcs[s]) * s2[j] : 0.f;
+            b2[z] = (row && s <= r) ? ex2(csr2 - vcs2[s]) * s2[j] : 0.f;
           }
           split2(b2[0], b2[1], vh[m], vl[m]);
         }
@@ -438,12 +438,27 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
     if (lane == 0) red[warp] = sp;
     __syncthreads();
     const float scal = red[0] + red[1] + red[2] + red[3] + red[4] + red[5] + red[6] + red[7];
-    if (tid == 0) {
-      float run = 0.f;
-      for (int l = len - 1; l >= 0; --l) {
-        run += vdcs[l] - vdl[l] * vxg[l] + (l == len - 1 ? scal : 0.f);
-        vdcs[l] = run;
+    // reverse cumsum of dcs over the chunk by warp 0: four tokens per lane, then a
+    // suffix scan of the lanes' totals
+    if (warp == 0) {
+      float d[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int l = 4 * lane + q;
+        d[q] = l < len ? vdcs[l] - vdl[l] * vxg[l] + (l == len - 1 ? scal : 0.f) : 0.f;
       }
+      d[2] += d[3];
+      d[1] += d[2];
+      d[0] += d[1];
+      float tot = d[0];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_down_sync(0xffffffffu, tot, o);
+        if (lane + o < 32) tot += u;
+      }
+      const float after = tot - d[0];  // everything in the lanes above this one
+#pragma unroll
+      for (int q = 0; q < 4; ++q) vdcs[4 * lane + q] = d[q] + after;
     }
     __syncthreads();
     float pA = 0.f, pb = 0.f;
