@@ -303,15 +303,16 @@ def run_step(args, w, rank, world, local, pg, hbm_peak, peak_kind):
         pg.destroy_process_group()
 
 
-def run_bwd(args, w, rank, world, local, pg, hbm_peak, peak_kind):
+def run_bwd(args, w, rank, world, local, pg, hbm_peak, tc_peak, peak_kind):
     """--op backward: ``ssd_backward`` over the workload (all gradients, fp32).
 
-    The backward runs on the CUDA cores, so its roofline is the fp32 FMA rate:
-    148 SMs x 128 lanes x 2 flops x 1965 MHz = 74.4 TFLOP/s.  Its algorithmic flops
-    per token and head, for chunks of Q = 64 tokens, are 2 Q (2 P + 3 N) (the
-    in-chunk products W, V, dC, dB, gB) + 8 N P (the state-sized products of dC, dB,
-    gB and the per-chunk cotangent sum) + 2 N P (the forward's chunk states,
-    recomputed).  L2 is flushed before every timed step.
+    Algorithmic flops per token and head, for chunks of Q tokens: 2 Q (2 P + 3 N)
+    (the in-chunk products W, V, dC, dB, gB) + 8 N P (the state-sized products of
+    dC, dB, gB and the per-chunk cotangent sum) + 2 N P (the forward's chunk states,
+    recomputed).  bf16 inputs with P = 64 and N = 64 or 128 take the tensor-core path
+    (Q = 128): its roofline is the measured bf16 tensor rate.  Every other shape runs
+    on the CUDA cores (Q = 64) against the fp32 FMA rate, 148 SMs x 128 lanes x 2 x
+    1965 MHz = 74.4 TFLOP/s.  L2 is flushed before every timed step.
     """
     import torch
 
@@ -359,9 +360,16 @@ def run_bwd(args, w, rank, world, local, pg, hbm_peak, peak_kind):
     ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
     ms = max_over_ranks(pg, ms)
     T = bsz * L
-    Q = 64
+    on_tc = w.dtype == "bf16" and P == 64 and N in (64, 128)
+    Q = 128 if on_tc else 64
     flops = float(T) * H * (2 * Q * (2 * P + 3 * N) + 10 * N * P)
-    peak = 148 * 128 * 2 * 1965e6 / 1e12
+    if on_tc:
+        bound, peak = "tensor", tc_peak
+        peak_source = (f"{peak_kind} bf16 tensor rate (MEASURED_PEAKS.json burst)" if peak_kind == "measured"
+                       else "fallback bf16 tensor rate")
+    else:
+        bound, peak = "alu", 148 * 128 * 2 * 1965e6 / 1e12
+        peak_source = "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"
     achieved = flops / (ms * 1e-3) / 1e12
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -380,7 +388,7 @@ def run_bwd(args, w, rank, world, local, pg, hbm_peak, peak_kind):
                          "scaled to the whole layer"}
     if rank == 0:
         line = {
-            "metric": "SSD chunked-scan backward (ssd_backward) Mtokens/s and % of fp32 FMA roofline",
+            "metric": "SSD chunked-scan backward (ssd_backward) Mtokens/s and % of roofline (tensor or fp32 FMA)",
             "value": T * world / (ms * 1e-3) / 1e6, "unit": "Mtokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -389,11 +397,12 @@ def run_bwd(args, w, rank, world, local, pg, hbm_peak, peak_kind):
                        "headdim": P, "dstate": N, "ngroups": G, "input_dtype": w.dtype,
                        "parallelism": f"dp{world} (independent replicas)",
                        "l2": "flushed before every timed step (512 MiB write, outside the events)"},
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None,
-                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
-                         "algorithmic_flops_per_launch": flops,
-                         "kernel": "kb_chunk + kb_chunk_dstate + kb_state_pass + the forward's state kernels"},
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "peak_source": peak_source,
+                         "algorithmic_flops_per_launch": flops, "chunk": Q,
+                         "kernel": ("kb_chunk_tc + kb_states_tc x2 + kb_state_pass + k_cumsum + k_state_pass"
+                                    if on_tc else
+                                    "kb_chunk + kb_chunk_dstate + kb_state_pass + the forward's state kernels")},
             "cpu_baseline": cpu, "e2e": None, "gpu_launches": 11 * args.steps, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -627,7 +636,7 @@ def main():
         run_cp(args, w, rank, world, local, pg, hbm_peak, peak_kind)
         return
     if args.op == "backward":
-        run_bwd(args, w, rank, world, local, pg, hbm_peak, peak_kind)
+        run_bwd(args, w, rank, world, local, pg, hbm_peak, tc_peak, peak_kind)
         return
     if args.op == "ext":
         run_ext(args, w, rank, world, local, pg, hbm_peak, peak_kind)
