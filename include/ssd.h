@@ -213,10 +213,13 @@ SSD_API int ssd_forward_host(ssd_handle_t h, const void* x, const void* dt, cons
  *   dx [batch, seqlen, H, P]; ddt [batch, seqlen, H]; dB, dC [batch, seqlen, G, N]
  *   (summed over the heads of each group); dA [H]; dD [H] and ddt_bias [H]
  *   (either may be NULL: not computed); dinitial_states [docs, H, N, P] or NULL.
- * It runs on the CUDA cores in fp32 with chunks of 64 tokens whatever chunk size
- * the forward used (the chunking changes only rounding).  dB, dC, dA, dD and
- * ddt_bias are sums of fp32 atomic additions, so their last bits can differ from
- * run to run.  Workspace grows in the handle as for ssd_forward.  Errors as for
+ * The chunk size is the backward's own, whatever the forward used (the chunking
+ * changes only rounding).  bf16 inputs and outputs with headdim 64, dstate 64 or
+ * 128 and 16-byte aligned x, B, C, dy, dx, dB and dC run on the tensor cores with
+ * 128-token chunks: bf16 operands, the in-chunk weighted matrices and the
+ * cotangent as hi + lo bf16 pairs, fp32 accumulation.  Everything else runs on the
+ * CUDA cores in fp32 with 64-token chunks.  dB, dC, dA, dD and ddt_bias are sums of
+ * fp32 atomic additions, so their last bits can differ from run to run.  Workspace grows in the handle as for ssd_forward.  Errors as for
  * ssd_forward; inputs need only element alignment.
  */
 SSD_API int ssd_backward(ssd_handle_t h, const void* x, const void* dt, const float* A,
