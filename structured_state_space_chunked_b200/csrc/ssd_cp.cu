@@ -129,9 +129,10 @@ __global__ void __launch_bounds__(256)
 // 128-token tiles); a persistent grid strides over the items.  Per item the CTA
 // writes its block of H_in once as a bf16 MN-major operand (state rows n are K).
 // Per tile: TMA brings the C tile and the y tile into shared memory, one thread
-// issues C H_in into TMEM (M = 128 tokens, N = Pc, K = dstate), each thread adds
-// exp(cs_t) times its accumulator row to its y row in shared memory, and a TMA
-// store writes the y tile back (rows past the slice are clipped by the store).
+// issues C H_in into TMEM (M = 128 tokens, N = Pc, K = dstate), two threads per token
+// row add exp(cs_t) times their halves of its accumulator row to its y row in shared
+// memory, and a TMA store writes the y tile back (rows past the slice are clipped by
+// the store).
 constexpr int kCorrTile = 128;
 struct CorrParams {
   int64_t L;
@@ -161,7 +162,7 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t ph, int* statu
   return true;
 }
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
     cp_correct_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
                          const __grid_constant__ CorrParams p) {
   using namespace tc;
@@ -176,7 +177,8 @@ __global__ void __launch_bounds__(128)
   const uint32_t c_bytes = (uint32_t)npanel * kPanel, y_bytes = (uint32_t)ypanels * kPanel;
   const uint32_t off_y = c_bytes, off_hb = c_bytes + y_bytes;
   const uint32_t hb_panel = (uint32_t)p.N * 128u;    // one 64-column panel of the state block
-  const int warp = threadIdx.x >> 5, r = threadIdx.x;
+  // 256 threads: threads r and r + 128 share token row r, each taking half the columns
+  const int warp = threadIdx.x >> 5, r = threadIdx.x & 127, half = threadIdx.x >> 7;
   const int nblk = p.P / p.Pc;
   const uint32_t full = su32(&bars[0]), done = su32(&bars[1]);
   const uint32_t tcols = (uint32_t)p.Pc;
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(128)
   const uint32_t tmem = tslot;
   const uint32_t id = idesc(128, p.Pc, 0, 1);
   const uint64_t dc = sdesc(sbase, 16, 1024), dh = sdesc(sbase + off_hb, hb_panel, 1024);
-  const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   uint32_t it = 0;  // tiles done by this CTA: the barriers' phase
   bool ok = true;
   for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(128)
     const int b = bh / p.H, h = bh % p.H, g = h / (p.H / p.G);
     // this block of H_in as bf16: row n, 64-column panels, 128-byte swizzle
     const float* hsrc = p.h_in + (int64_t)bh * p.N * p.P + pb * p.Pc;
-    for (int i = r; i < p.N * (p.Pc / 8); i += blockDim.x) {
+    for (int i = threadIdx.x; i < p.N * (p.Pc / 8); i += blockDim.x) {
       const int n = i / (p.Pc / 8), c8 = i % (p.Pc / 8);
       const float4 u = *reinterpret_cast<const float4*>(hsrc + (int64_t)n * p.P + 8 * c8);
       const float4 v = *reinterpret_cast<const float4*>(hsrc + (int64_t)n * p.P + 8 * c8 + 4);
@@ -243,7 +245,7 @@ __global__ void __launch_bounds__(128)
       tc_fence_after();
       const int64_t t = (int64_t)t0 + r;
       const float e = (ok && t < p.L) ? expf(p.cs[((int64_t)b * p.L + t) * p.H + h]) : 0.f;
-      for (int c0 = 0; c0 < p.Pc; c0 += 32) {
+      for (int c0 = half * (p.Pc / 2); c0 < (half + 1) * (p.Pc / 2); c0 += 32) {
         float acc[32];
         tc_ld32(ta + c0, acc);
         tc_wait_ld();
@@ -435,7 +437,7 @@ extern "C" SSD_API int ssd_cp_correct(const ssd_desc_t* desc, const void* C, con
     if (cudaFuncSetAttribute(ssd::cp_correct_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return SSD_ERR_CUDA;
-    ssd::cp_correct_tc_kernel<<<grid, 128, smem, st>>>(tm_c, tm_y, p);
+    ssd::cp_correct_tc_kernel<<<grid, 256, smem, st>>>(tm_c, tm_y, p);
     return ssd::launch_rc();
   }
   const size_t smem = sizeof(float) * ((size_t)d.dstate * d.headdim + (size_t)ssd::kCorrTok * d.dstate);
