@@ -27,6 +27,9 @@
 //   kb_chunk         every per-token gradient of one (chunk, head) from 64 x 64 tiles
 //                    in shared memory; dB and dC add over the heads of a group
 //                    (fp32 atomics), dA, dD and ddt_bias over chunks.
+// For bf16 inputs with P = 64 and N = 64 or 128 (bwd_tc_eligible) the chunks are 128
+// tokens long and ssd_bwd_tc.cu takes over the products: kb_chunk_tc in place of
+// kb_chunk and, for N = 128, kb_states_tc in place of the two chunk-state products.
 #include <cuda_runtime.h>
 
 #include "ssd_bwd.h"
