@@ -75,6 +75,32 @@ __global__ void cp_combine_kernel(int r, int nranks, int64_t BH, int64_t NP, con
   (void)nranks;
 }
 
+// The same, four consecutive state elements per thread with 16-byte accesses (N P a
+// multiple of 4 and every array 16-byte aligned); every rank's load is issued before
+// the Horner updates that use it.
+__device__ __forceinline__ float4 f4_fma(float a, float4 x, float4 y) {
+  return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
+}
+__global__ void cp_combine4_kernel(int r, int64_t BH, int64_t NP, const float4* S_all, const float* ld_all,
+                                   const float4* init, float4* h_in, float4* final_states) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // float4 index
+  const int64_t NP4 = NP / 4;
+  if (i >= BH * NP4) return;
+  const int64_t bh = i / NP4;
+  float4 hv = init ? __ldg(init + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  int k = 0;
+  for (; k + 4 <= r; k += 4) {
+    float4 s[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) s[u] = __ldg(S_all + (k + u) * BH * NP4 + i);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) hv = f4_fma(expf(ld_all[(k + u) * BH + bh]), hv, s[u]);
+  }
+  for (; k < r; ++k) hv = f4_fma(expf(ld_all[k * BH + bh]), hv, __ldg(S_all + k * BH * NP4 + i));
+  if (h_in) h_in[i] = hv;
+  if (final_states) final_states[i] = f4_fma(expf(ld_all[r * BH + bh]), hv, __ldg(S_all + r * BH * NP4 + i));
+}
+
 // y[b, t, h, :] += exp(cs[b, t, h]) C[b, t, g, :] H_in[b, h]: one CTA per (b, h, 64 tokens);
 // the state in shared memory, 4 tokens x 4 columns per thread.
 constexpr int kCorrTok = 64;
@@ -361,8 +387,17 @@ extern "C" SSD_API int ssd_cp_combine(const ssd_desc_t* desc, int rank, int nran
   if (BH == 0) return SSD_OK;
   if (!local_final_all || !logdecay_all || (!h_in && !final_states)) return SSD_ERR_INVALID_ARG;
   const int64_t n = BH * NP;
-  ssd::cp_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0,
-                           reinterpret_cast<cudaStream_t>(stream)>>>(
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (NP % 4 == 0 && ssd::aligned(local_final_all, 16) && ssd::aligned(initial_states, 16) &&
+      ssd::aligned(h_in, 16) && ssd::aligned(final_states, 16)) {
+    const int64_t n4 = n / 4;
+    ssd::cp_combine4_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(
+        rank, BH, NP, reinterpret_cast<const float4*>(local_final_all), logdecay_all,
+        reinterpret_cast<const float4*>(initial_states), reinterpret_cast<float4*>(h_in),
+        reinterpret_cast<float4*>(final_states));
+    return ssd::launch_rc();
+  }
+  ssd::cp_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
       rank, nranks, BH, NP, local_final_all, logdecay_all, initial_states, h_in, final_states);
   return ssd::launch_rc();
 }
