@@ -133,3 +133,29 @@ def test_feature_map_dims_without_a_gpu():
     assert [ssd.feature_map_dim(k, 8) for k in range(5)] == [8, 8, 8, 73, 64]
     assert ssd.lib().ssd_feature_map_dim(7, 8) == -1
     assert ssd.lib().ssd_forward_ext(None, *([None] * 7), 64, None, 0, 1, 0, None, None, None) == -1
+
+
+def test_context_parallel_entries_validate_their_arguments_without_a_gpu():
+    # every check below returns before the device is touched
+    L = ssd.lib()
+    d = ssd.make_desc(2, 128, 4, 64, 128, 1, torch.bfloat16)
+    packed = ssd.make_desc(1, 128, 4, 64, 128, 1, torch.bfloat16, max_docs=3)  # batch mode only
+    bad_g = ssd.make_desc(2, 128, 3, 64, 128, 2, torch.bfloat16)
+    empty = ssd.make_desc(0, 128, 4, 64, 128, 1, torch.bfloat16)
+    assert L.ssd_cp_logdecay(None, None, None, None, None, None, None) == -1
+    assert L.ssd_cp_logdecay(ctypes.byref(packed), None, None, None, None, None, None) == -1
+    assert L.ssd_cp_logdecay(ctypes.byref(bad_g), None, None, None, None, None, None) == -1
+    assert L.ssd_cp_logdecay(ctypes.byref(d), None, None, None, None, None, None) == -1   # null arrays
+    assert L.ssd_cp_logdecay(ctypes.byref(empty), None, None, None, None, None, None) == 0
+    for rank, nranks in ((2, 2), (-1, 2), (0, 0)):
+        assert L.ssd_cp_combine(ctypes.byref(d), rank, nranks, None, None, None, None, None, None) == -1
+    assert L.ssd_cp_combine(ctypes.byref(d), 0, 2, None, None, None, None, None, None) == -1
+    assert L.ssd_cp_correct(ctypes.byref(d), None, None, None, None, None, None) == -1
+
+
+def test_forward_ext_and_backward_refuse_bad_options_without_a_gpu():
+    L = ssd.lib()
+    # unknown feature map, and normalize outside {0, 1}: refused by the missing handle first
+    assert L.ssd_forward_ext(None, *([None] * 7), 64, None, 0, 9, 0, None, None, None) == -1
+    assert L.ssd_forward_ext(None, *([None] * 7), 64, None, 0, 1, 2, None, None, None) == -1
+    assert ssd.lib().ssd_feature_map_dim(ssd.SSD_FMAP_BASED, 0) == -1
