@@ -7,7 +7,7 @@ cumulative decay, the diagonal blocks, the chunk states, the state passing and
 the outputs), inputs resident in HBM.  Each rank runs the full per-GPU workload
 (weak scaling; ranks share nothing, the work has no data-path collective).
 L2 is flushed (a 512 MiB write) before every timed step, outside the timed
-events.  Times are CUDA events on the launching stream, summed over the K
+events.  Times are CUDA events on the launching stream, the median of the K
 steps, max over ranks.  ``--impl reference`` times the float64 oracle on the
 host cores on a bounded sample of the same workload (rank 0 only).
 """
@@ -29,7 +29,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "SSD chunked-scan fwd Mtokens/s and % of roofline (HBM or tensor pipe)"
-DEFAULT_WORKLOAD = "mamba2_130m_layer_b4_L2048"
+DEFAULT_WORKLOAD = "long_L65536_H64_P128_N256_G8"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -261,7 +261,7 @@ def run_step(args, w, rank, world, local, pg, hbm_peak, peak_kind):
     clk.region(t_wall0, t_wall1)
     time.sleep(0.1)
     clocks = clk.stop()
-    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    ms = statistics.median(a.elapsed_time(b) for a, b in zip(starts, ends))
     ms = max_over_ranks(pg, ms)
     ein = 2 if w.dtype == "bf16" else 4
     byts = bsz * H * (8 * N * P + 2 * P * ein + ein) + 2 * bsz * G * N * ein + 12 * H
@@ -357,7 +357,7 @@ def run_bwd(args, w, rank, world, local, pg, hbm_peak, tc_peak, peak_kind):
     clk.region(t_wall0, t_wall1)
     time.sleep(0.1)
     clocks = clk.stop()
-    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    ms = statistics.median(a.elapsed_time(b) for a, b in zip(starts, ends))
     ms = max_over_ranks(pg, ms)
     T = bsz * L
     on_tc = w.dtype == "bf16" and P == 64 and N in (64, 128)
@@ -465,7 +465,7 @@ def run_ext(args, w, rank, world, local, pg, hbm_peak, peak_kind):
     clk.region(t_wall0, t_wall1)
     time.sleep(0.1)
     clocks = clk.stop()
-    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    ms = statistics.median(a.elapsed_time(b) for a, b in zip(starts, ends))
     ms = max_over_ranks(pg, ms)
     es = 2 if w.dtype == "bf16" else 4
     T = bsz * L
@@ -559,9 +559,9 @@ def run_cp(args, w, rank, world, local, pg, hbm_peak, peak_kind):
     clk.region(t_wall0, t_wall1)
     time.sleep(0.1)
     clocks = clk.stop()
-    ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    ms = statistics.median(a.elapsed_time(b) for a, b in zip(starts, ends))
     ms = max_over_ranks(pg, ms)
-    corr_ms = sum(a.elapsed_time(b) for a, b in corr_ev) / args.steps
+    corr_ms = statistics.median(a.elapsed_time(b) for a, b in corr_ev)
     on_tc = w.dtype == "bf16" and P % 64 == 0 and P <= 256 and N % 64 == 0 and N <= 256
     ein = 2 if w.dtype == "bf16" else 4
     T = bsz * L
@@ -619,8 +619,8 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=256,
                     help="sequences per ssd_step call (--op step)")
     args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
+    # at least 10 untimed warm-up steps (the reported "warmup" is the count run)
+    args.warmup = max(args.warmup, 10)
 
     import torch
     from structured_state_space_chunked_b200 import inputs as I
@@ -731,7 +731,8 @@ def main():
     st = h.status()
     if st != 0:
         raise SystemExit(f"device status {st} in the timed region")
-    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    # the median step (CUDA events), then the max over ranks
+    ms = statistics.median(s.elapsed_time(e) for s, e in zip(starts, ends))
     ms = max_over_ranks(pg, ms)
     tokens_all = w.tokens * world
     value = tokens_all / (ms * 1e-3) / 1e6

@@ -372,7 +372,8 @@ SSD_API int ssd_cp_correct(const ssd_desc_t* desc, const void* C, const float* c
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture.  All calls on a device share the one array and the previous
+ * any stream capture.  The address is kept for the life of the process, so a
+ * device reset (cudaDeviceReset) between calls is not supported.  All calls on a device share the one array and the previous
  * call's contents stay in it (nothing needs to start at zero), so calls whose GPU
  * work overlaps -- on different streams without ordering -- race and must be
  * serialised by the caller.

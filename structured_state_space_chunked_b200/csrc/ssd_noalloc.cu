@@ -14,7 +14,9 @@
 // Host code must not use `ssd_noalloc_scratch` as a pointer: on the host that name
 // is only a stand-in for the device symbol.  Its device address is looked up once
 // per device with cudaGetSymbolAddress (the first call on a device does this, with
-// that device current) and is then passed to the kernels.
+// that device current) and is then passed to the kernels.  The address is kept
+// until the process exits: a device reset between calls is not supported (the
+// module would be reloaded and the array could move).
 //
 // Every call on a device uses the same array, and it keeps whatever the previous
 // call left in it.  Nothing in it has to start at zero: each call's kernels write

@@ -504,7 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every MMA this thread issued has completed once TEARDOWN fires
       tc_commit(bar(TEARDOWN));
-      wait_bar(bar(TEARDOWN), 0, abort_flag, kp.status);
+      // bounded by time only: TMEM is freed below, so no MMA may still run then
+      if (!wait_drain(bar(TEARDOWN), 0, 2000000000ull)) set_status(kp.status, SSD_ERR_TIMEOUT);
     }
   } else {
     // ==================== epilogue group w: every other tile, end to end ====================

@@ -40,6 +40,16 @@ __device__ __forceinline__ uint64_t globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+// Wait for a phase bounded by time only.  Used before freeing what issued work
+// still touches (TMEM under in-flight MMAs, shared memory under in-flight TMA
+// loads): no abort flag may cut this wait short.  False when it ran out.
+__device__ __forceinline__ bool wait_drain(uint32_t a, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(a, parity)) {
+    if (globaltimer() - t0 > limit_ns) return false;
+  }
+  return true;
+}
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

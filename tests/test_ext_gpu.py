@@ -17,29 +17,43 @@ from tests.parity_util import TOL, make, rel_err, to_np
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    # dtype, batch, seqlen, H, P, N, G, feature map, normalize, varlen tokens
-    ("bf16", 2, 300, 4, 64, 128, 1, ssd.SSD_FMAP_SILU, False, 0),
-    ("bf16", 2, 300, 4, 64, 64, 2, ssd.SSD_FMAP_RELU, True, 0),
-    ("fp32", 1, 200, 3, 16, 8, 1, ssd.SSD_FMAP_BASED, True, 0),
-    ("bf16", 1, 257, 2, 64, 8, 1, ssd.SSD_FMAP_REBASED, True, 0),
-    ("bf16", 1, 0, 2, 64, 16, 1, ssd.SSD_FMAP_BASED, True, 1000),
-    ("fp32", 2, 100, 2, 32, 16, 1, ssd.SSD_FMAP_NONE, True, 0),
-    ("fp32", 2, 130, 2, 32, 16, 2, ssd.SSD_FMAP_RELU, False, 0),
+    # dtype, batch, seqlen, H, P, N, G, feature map, normalize, varlen tokens, chunk
+    # chunk 64: the numerator runs on the CUDA-core path (the tensor-core kernel
+    # needs chunks of a multiple of 128 tokens)
+    ("bf16", 2, 300, 4, 64, 128, 1, ssd.SSD_FMAP_SILU, False, 0, 64),
+    ("bf16", 2, 300, 4, 64, 64, 2, ssd.SSD_FMAP_RELU, True, 0, 64),
+    ("fp32", 1, 200, 3, 16, 8, 1, ssd.SSD_FMAP_BASED, True, 0, 64),
+    ("bf16", 1, 257, 2, 64, 8, 1, ssd.SSD_FMAP_REBASED, True, 0, 64),
+    ("bf16", 1, 0, 2, 64, 16, 1, ssd.SSD_FMAP_BASED, True, 1000, 64),
+    ("fp32", 2, 100, 2, 32, 16, 1, ssd.SSD_FMAP_NONE, True, 0, 64),
+    ("fp32", 2, 130, 2, 32, 16, 2, ssd.SSD_FMAP_RELU, False, 0, 64),
+    # chunk 256, bf16, mapped dstate a multiple of 16: the numerator runs on the
+    # tensor cores over the mapped B and C (the configuration the benchmark times)
+    ("bf16", 2, 600, 4, 64, 64, 1, ssd.SSD_FMAP_SILU, False, 0, 256),
+    ("bf16", 2, 520, 4, 64, 128, 2, ssd.SSD_FMAP_RELU, True, 0, 256),
+    ("bf16", 1, 700, 2, 64, 8, 1, ssd.SSD_FMAP_REBASED, True, 0, 256),
+    ("bf16", 1, 0, 4, 64, 8, 1, ssd.SSD_FMAP_REBASED, True, 1500, 256),
 ]
-IDS = ["silu-tc", "relu-norm-tc", "based-norm-simt", "rebased-norm-tc", "based-norm-packed",
-       "none-norm", "relu-fp32"]
+IDS = ["silu-simt", "relu-norm-simt", "based-norm-simt-fp32", "rebased-norm-simt",
+       "based-norm-packed-simt", "none-norm-fp32", "relu-fp32",
+       "silu-tc", "relu-norm-tc", "rebased-norm-tc", "rebased-norm-packed-tc"]
 
 
 @pytest.mark.parametrize("case", CASES, ids=IDS)
 def test_forward_ext_matches_oracle(case):
-    dtype, b, L, H, P, N, G, fmap, norm, vt = case
-    w = I.random_small(900 + N + P, dtype, b, L, H, P, N, G, 64, "zero", vt)
+    dtype, b, L, H, P, N, G, fmap, norm, vt, Q = case
+    w = I.random_small(900 + N + P, dtype, b, L, H, P, N, G, Q, "zero", vt)
     inp = make(w)
     bsz, Lr = inp["x"].shape[:2]
     max_docs = 0 if inp["cu_seqlens"] is None else inp["cu_seqlens"].numel() - 1
     h = ssd.SSD(bsz, Lr, H, P, N, G, w.torch_dtype, max_docs=max_docs)
+    # the path the numerator takes is the plain forward's path at the mapped dstate
+    n2 = ssd.feature_map_dim(fmap, N)
+    mapped = ssd.make_desc(bsz, Lr, H, P, n2, G, w.torch_dtype, max_docs=max_docs)
+    want = ssd.SSD_PATH_TC if Q == 256 else ssd.SSD_PATH_SIMT
+    assert ssd.plan(mapped, Q, max_docs).path == want
     y, fin = h.forward_ext(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
-                           inp["dt_bias"], 64, feature_map=fmap, normalize=norm,
+                           inp["dt_bias"], Q, feature_map=fmap, normalize=norm,
                            cu_seqlens=inp["cu_seqlens"])
     assert h.status() == 0
     torch.cuda.synchronize()
@@ -71,6 +85,17 @@ def test_unknown_feature_map_is_refused():
     h = ssd.SSD(1, 64, 2, 64, 64, 1, torch.bfloat16)
     with pytest.raises(ssd.SSDError):
         h.forward_ext(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], feature_map=9)
+
+
+def test_normalize_outside_zero_one_is_refused():
+    w = I.random_small(2, "bf16", 1, 64, 2, 64, 64, 1, 64)
+    inp = make(w)
+    h = ssd.SSD(1, 64, 2, 64, 64, 1, torch.bfloat16)
+    y = torch.empty_like(inp["x"])
+    rc = ssd.lib().ssd_forward_ext(h._h, *(ssd._ptr(inp[k]) for k in ("x", "dt", "A", "B", "C")),
+                                   None, None, 64, None, 0, ssd.SSD_FMAP_RELU, 2, ssd._ptr(y),
+                                   None, None)
+    assert rc == -1
 
 
 def test_forward_ext_bad_cu_seqlens_sets_status():

@@ -153,9 +153,11 @@ def test_context_parallel_entries_validate_their_arguments_without_a_gpu():
     assert L.ssd_cp_correct(ctypes.byref(d), None, None, None, None, None, None) == -1
 
 
-def test_forward_ext_and_backward_refuse_bad_options_without_a_gpu():
+def test_forward_ext_refuses_a_missing_handle_and_feature_map_dim_checks_without_a_gpu():
+    # (the option checks behind a valid handle are GPU tests in test_ext_gpu.py)
     L = ssd.lib()
-    # unknown feature map, and normalize outside {0, 1}: refused by the missing handle first
-    assert L.ssd_forward_ext(None, *([None] * 7), 64, None, 0, 9, 0, None, None, None) == -1
-    assert L.ssd_forward_ext(None, *([None] * 7), 64, None, 0, 1, 2, None, None, None) == -1
-    assert ssd.lib().ssd_feature_map_dim(ssd.SSD_FMAP_BASED, 0) == -1
+    assert L.ssd_forward_ext(None, *([None] * 7), 64, None, 0, 1, 0, None, None, None) == -1
+    assert L.ssd_feature_map_dim(9, 16) == -1          # unknown feature map
+    assert L.ssd_feature_map_dim(ssd.SSD_FMAP_BASED, 0) == -1
+    assert L.ssd_feature_map_dim(ssd.SSD_FMAP_BASED, 8) == 1 + 8 + 64
+    assert L.ssd_feature_map_dim(ssd.SSD_FMAP_REBASED, 8) == 64

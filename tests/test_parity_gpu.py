@@ -110,28 +110,41 @@ def test_mamba2_130m_layer_full_oracle():
     check(w, inp, y, fin)
 
 
-def test_mamba2_2p7b_layer_sampled_heads():
+def test_mamba2_2p7b_layer_all_heads():
     w = I.workload("mamba2_2p7b_layer_b8_L4096")
     inp = make(w)
     y, fin, _ = gpu_run(w, inp)
-    check(w, inp, y, fin, heads=[0, 37, 79])
+    check(w, inp, y, fin)
 
 
-@pytest.mark.parametrize("w", [w for w in I.workloads() if w.name.startswith("long_")],
-                         ids=lambda w: w.name)
-def test_long_sequence_sampled_heads(w):
+LONG = [w for w in I.workloads() if w.name.startswith("long_")]
+
+
+@pytest.mark.parametrize("w", [w for w in LONG if w.seqlen <= 16384], ids=lambda w: w.name)
+def test_long_sequence_all_heads(w):
     inp = make(w)
     y, fin, h = gpu_run(w, inp)
-    check(w, inp, y, fin, heads=[5, 60])
+    check(w, inp, y, fin)
     del y, fin, inp, h
     torch.cuda.empty_cache()
 
 
-def test_varlen_packed_documents():
+@pytest.mark.parametrize("w", [w for w in LONG if w.seqlen > 16384], ids=lambda w: w.name)
+def test_long_sequence_65536_sampled_heads(w):
+    # host memory bounds the float64 reference here: heads from both halves of the
+    # head range and of two different B/C groups, every token and state element
+    inp = make(w)
+    y, fin, h = gpu_run(w, inp)
+    check(w, inp, y, fin, heads=[0, 5, 33, 60, 63])
+    del y, fin, inp, h
+    torch.cuda.empty_cache()
+
+
+def test_varlen_packed_documents_all_heads():
     w = I.workload("varlen_32k_H32_P64_N128")
     inp = make(w)
     y, fin, _ = gpu_run(w, inp)
-    check(w, inp, y, fin, heads=[0, 13, 31])
+    check(w, inp, y, fin)
 
 
 @pytest.mark.parametrize("path", PATHS, ids=["simt", "tc"])

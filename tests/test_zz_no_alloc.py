@@ -6,8 +6,9 @@ library.
 
 The test calls it through the C ABI twice in a row (different problems, so the
 second call runs on whatever the first left in the shared scratch) and checks
-each output against the existing ssd_forward entry point within the parity
-tolerance, then checks that a problem too big for the array is refused.  This
+each output against the existing ssd_forward entry point and against the
+float64 oracle, within the parity tolerance, then checks that a problem too big
+for the array is refused.  This
 file is collected last so that a stop-at-first-failure run has already run every
 other test."""
 
@@ -18,7 +19,7 @@ import torch
 
 from structured_state_space_chunked_b200 import inputs as I
 from structured_state_space_chunked_b200 import ssd
-from tests.parity_util import TOL, make, rel_err, to_np
+from tests.parity_util import TOL, make, oracle_run, rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -71,6 +72,10 @@ def test_noalloc_matches_ssd_forward_on_two_calls_in_a_row():
         tol = TOL[w.dtype]
         assert rel_err(to_np(y), to_np(y_ref)) <= tol
         assert rel_err(to_np(fin), to_np(fin_ref)) <= tol
+        # and directly against the float64 oracle on the same inputs
+        y_or, fin_or = oracle_run(inp)
+        assert rel_err(to_np(y), y_or) <= tol
+        assert rel_err(to_np(fin), fin_or) <= tol
 
 
 def test_noalloc_refuses_a_problem_larger_than_its_scratch():
