@@ -18,6 +18,8 @@ struct ssd_handle_s {
   int num_sms;
   int force_path;
   int tc_unit_columns;  // 64 or 128
+  unsigned long long wait_ns;  // bound of every device-side wait of the tensor-core kernel
+  int force_timeout;    // 1: the tensor-core kernel's first epilogue wait runs out (test)
   int* status;          // device status word (first error code, 0 = ok)
   void* ws;             // stream-ordered workspace
   size_t ws_bytes;
@@ -79,6 +81,14 @@ int cuda_rc(cudaError_t e) {
   return SSD_ERR_CUDA;
 }
 
+ssd::TcOpts tc_opts(const ssd_handle_s* h) {
+  ssd::TcOpts o;
+  o.unit_columns = h->tc_unit_columns;
+  o.wait_ns = h->wait_ns;
+  o.stall = h->force_timeout;
+  return o;
+}
+
 }  // namespace
 
 extern "C" {
@@ -135,6 +145,8 @@ int ssd_create(const ssd_desc_t* desc, ssd_handle_t* out) {
   h->num_sms = sms;
   h->force_path = SSD_PATH_AUTO;
   h->tc_unit_columns = 64;
+  h->wait_ns = 2000000000ull;
+  h->force_timeout = 0;
   cudaError_t e = cudaMalloc(&h->status, sizeof(int) * 4);
   if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int) * 4);
   if (e != cudaSuccess) {
@@ -157,6 +169,16 @@ int ssd_set_option(ssd_handle_t h, int option, int value) {
   if (option == SSD_OPT_TC_UNIT_COLUMNS) {
     if (value != 64 && value != 128) return SSD_ERR_INVALID_ARG;
     h->tc_unit_columns = value;
+    return SSD_OK;
+  }
+  if (option == SSD_OPT_WAIT_LIMIT_US) {
+    if (value < 1 || value > 60000000) return SSD_ERR_INVALID_ARG;
+    h->wait_ns = 1000ull * (unsigned long long)value;
+    return SSD_OK;
+  }
+  if (option == SSD_OPT_TEST_FORCE_TIMEOUT) {
+    if (value != 0 && value != 1) return SSD_ERR_INVALID_ARG;
+    h->force_timeout = value;
     return SSD_OK;
   }
   return SSD_ERR_INVALID_ARG;
@@ -206,7 +228,7 @@ int ssd_forward(ssd_handle_t h, const void* x, const void* dt, const float* A, c
   ssd::Args a{x, dt, A, B, C, D, dt_bias, initial_states, cu_seqlens, y, final_states};
   cudaError_t e;
   if (path == SSD_PATH_TC) {
-    e = ssd::tc_forward(g, a, h->ws, h->status, stream, h->num_sms, h->tc_unit_columns);
+    e = ssd::tc_forward(g, a, h->ws, h->status, stream, h->num_sms, tc_opts(h));
   } else {
     ssd::SimtWorkspace ws;
     ssd::simt_carve_workspace(g, h->ws, &ws);
@@ -339,7 +361,7 @@ int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* 
   ssd::Args a{x, dt, A, B2, C2, normalize ? nullptr : D, dt_bias, nullptr, cu_seqlens, y, final_states};
   if (e == cudaSuccess) {
     if (path == SSD_PATH_TC) {
-      e = ssd::tc_forward(g, a, fws, h->status, stream, h->num_sms, h->tc_unit_columns);
+      e = ssd::tc_forward(g, a, fws, h->status, stream, h->num_sms, tc_opts(h));
     } else {
       ssd::SimtWorkspace ws;
       ssd::simt_carve_workspace(g, fws, &ws);

@@ -75,12 +75,22 @@ cudaError_t simt_forward(const Geom& g, const Args& a, const SimtWorkspace& ws, 
                          cudaStream_t stream);
 
 // ---- tensor-core (tcgen05) path -------------------------------------------------
+// Launch options of the tensor-core forward (handle options of ssd_set_option).
+struct TcOpts {
+  int unit_columns = 64;                      // 64 or 128 (ssd_tc_wide.cu)
+  unsigned long long wait_ns = 2000000000ull; // bound of every device-side wait
+  int stall = 0;                              // 1: forced-timeout test (ssd_tc2.cu)
+};
 bool tc_supported(const Geom& g, const Args* a);
 int tc_units(const Geom& g);
 int tc_kernels(const Geom& g);
 size_t tc_workspace_bytes(const Geom& g);
 cudaError_t tc_forward(const Geom& g, const Args& a, void* workspace, int* status,
-                       cudaStream_t stream, int num_sms, int unit_columns);
+                       cudaStream_t stream, int num_sms, const TcOpts& opts);
+// the kernel with the state chain in registers (ssd_tc2.cu): N <= 128
+bool tc2_supported(const Geom& g);
+cudaError_t tc2_forward(const Geom& g, const Args& a, int* status, cudaStream_t stream, int num_sms,
+                        unsigned long long wait_ns, int stall);
 // 128-column units (ssd_tc_wide.cu): tc_forward with unit_columns == 128
 bool tc_wide_supported(const Geom& g);
 int tc_wide_units(const Geom& g);

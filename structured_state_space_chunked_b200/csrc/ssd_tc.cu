@@ -800,8 +800,9 @@ int tc_kernels(const Geom&) { return 1; }
 size_t tc_workspace_bytes(const Geom&) { return 256; }
 
 cudaError_t tc_forward(const Geom& g, const Args& a, void*, int* status, cudaStream_t stream,
-                       int num_sms, int unit_columns) {
-  if (unit_columns == 128) return tc_wide_forward(g, a, status, stream, num_sms);
+                       int num_sms, const TcOpts& opts) {
+  if (opts.unit_columns == 128) return tc_wide_forward(g, a, status, stream, num_sms);
+  if (tc2_supported(g)) return tc2_forward(g, a, status, stream, num_sms, opts.wait_ns, opts.stall);
   CUtensorMap tx, tb, tc;
   const cuuint64_t T = (cuuint64_t)g.tokens;
   {

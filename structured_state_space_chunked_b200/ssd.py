@@ -21,6 +21,8 @@ SSD_F32, SSD_BF16 = 0, 1
 SSD_PATH_AUTO, SSD_PATH_SIMT, SSD_PATH_TC = -1, 0, 1
 SSD_OPT_FORCE_PATH = 1
 SSD_OPT_TC_UNIT_COLUMNS = 2
+SSD_OPT_WAIT_LIMIT_US = 3
+SSD_OPT_TEST_FORCE_TIMEOUT = 4
 ERRORS = {
     0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3: "SSD_ERR_CUDA",
     -4: "SSD_ERR_TIMEOUT", -5: "SSD_ERR_OOM", -6: "SSD_ERR_BAD_SEQLENS",
@@ -173,6 +175,18 @@ class SSD:
     def tc_unit_columns(self, cols: int) -> None:
         """Column width (64 or 128) of the tensor-core kernel's work units."""
         rc = lib().ssd_set_option(self._h, SSD_OPT_TC_UNIT_COLUMNS, int(cols))
+        if rc:
+            raise SSDError(rc, "ssd_set_option")
+
+    def wait_limit_us(self, us: int) -> None:
+        """Bound (microseconds) of every device-side wait of the tensor-core kernel."""
+        rc = lib().ssd_set_option(self._h, SSD_OPT_WAIT_LIMIT_US, int(us))
+        if rc:
+            raise SSDError(rc, "ssd_set_option")
+
+    def force_timeout(self, on: bool) -> None:
+        """Failure-path test: make the tensor-core kernel's first wait run out."""
+        rc = lib().ssd_set_option(self._h, SSD_OPT_TEST_FORCE_TIMEOUT, int(bool(on)))
         if rc:
             raise SSDError(rc, "ssd_set_option")
 
