@@ -40,6 +40,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "ssd_internal.h"
 #include "tc_common.cuh"
 
@@ -411,16 +413,76 @@ __global__ void __launch_bounds__(kThreads, 1)
     // A non-blocking event loop over four in-order streams: dS (feeds the state
     // chain), Yoff (left factors), C B^T, Ydiag.  A B/C slot is released once the
     // three products that read it (dS, Yoff, C B^T) are issued.  The whole warp runs
-    // the loop with warp-uniform decisions; one elected lane issues each instruction.
+    // the loop with warp-uniform decisions and lane 0 issues each instruction.  Each
+    // product is issued by a path specialised on the tile's parity, so every operand
+    // is a loop-invariant base plus a compile-time offset.
     {
       constexpr uint32_t ID_CB = idesc(128, 128, 0, 0);    // Z = C B^T, both K-major
       constexpr uint32_t ID_YOFF = idesc(128, kPT, 0, 1);  // Yoff = C Hb, Hb MN-major
       constexpr uint32_t ID_ST = idesc(128, kPT, 1, 1);    // dS = B^T XW, both MN-major
       constexpr uint32_t ID_YD = idesc(128, kPT, 0, 1);    // Ydiag = M X, M in TMEM
-      auto bc_of = [&](uint32_t j) { return sbase + C::OFF_BC + (j % C::BS) * C::BC_BYTES; };
+      // loop-invariant descriptor bases
+      const uint64_t d_bc0 = sdesc(sbase + C::OFF_BC, 16, 1024);        // K-major B (slot 0)
+      const uint64_t d_bcm0 = sdesc(sbase + C::OFF_BC, kPanel, 1024);   // MN-major B (slot 0)
+      const uint64_t d_x0 = sdesc(sbase + C::OFF_X, kPanel, 1024);
+      const uint64_t d_xw0 = sdesc(sbase + C::OFF_XW, kPanel, 1024);
+      const uint64_t d_hb0 = sdesc(sbase + C::OFF_HB, C::HB_BYTES, 1024);
+      const uint32_t tm = tmem;
       auto tst = [&](int b, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_test(bar(b), parity));
       };
+      // w: parity of the tile; slot offsets of the rings follow from it
+      auto issue_ds = [&](auto W) {
+        constexpr uint32_t w = decltype(W)::value;
+        constexpr uint32_t bs = C::BS == 2 ? w : 0, ds = C::DSB == 2 ? w : 0;
+        const uint64_t dbm = d_bcm0 + ((bs * C::BC_BYTES) >> 4);
+        const uint64_t dxw = d_xw0 + ((w * kPanel) >> 4);
+        const uint32_t dcol = tm + C::COL_DS + ds * NT * kPT;
+#pragma unroll
+        for (int mt = 0; mt < NT; ++mt)
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            tc_mma_w(dcol + mt * kPT, dbm + ((2 * mt * kPanel + kk * 2048) >> 4),
+                     dxw + ((kk * 2048) >> 4), ID_ST, NT == 2 || kk > 0);
+        tc_commit_w(bar(DS_DONE0 + w));
+      };
+      auto issue_yo = [&](auto W) {
+        constexpr uint32_t w = decltype(W)::value;
+        constexpr uint32_t bs = C::BS == 2 ? w : 0, hs = C::HBS == 2 ? w : 0;
+        const uint64_t dc = d_bc0 + ((bs * C::BC_BYTES + C::BC1_BYTES) >> 4);
+        const uint64_t dhb = d_hb0 + ((hs * C::HB_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < C::NPAD / 16; ++kk)
+          tc_mma_w(tm + C::COL_YO + w * kPT, dc + (((kk >> 2) * kPanel + (kk & 3) * 32) >> 4),
+                   dhb + ((kk * 2048) >> 4), ID_YOFF, kk > 0);
+        tc_commit_w(bar(YO_DONE0 + w));
+      };
+      auto issue_cb = [&](auto W) {
+        constexpr uint32_t w = decltype(W)::value;
+        constexpr uint32_t bs = C::BS == 2 ? w : 0;
+        const uint64_t db = d_bc0 + ((bs * C::BC_BYTES) >> 4);
+        const uint64_t dc = db + (C::BC1_BYTES >> 4);
+#pragma unroll
+        for (int kk = 0; kk < C::NPAD / 16; ++kk) {
+          const uint64_t off = ((kk >> 2) * kPanel + (kk & 3) * 32) >> 4;
+          tc_mma_w(tm + C::COL_Z + w * 128, dc + off, db + off, ID_CB, kk > 0);
+        }
+        tc_commit_w(bar(CB_DONE0 + w));
+      };
+      auto issue_yd = [&](auto W) {
+        // Ydiag = M X_j : K = tokens.  M sits in TMEM as bf16 pairs (the 16 tokens of
+        // K step kk in columns 8kk..8kk+7 of the Z buffer); Ydiag goes next to it
+        constexpr uint32_t w = decltype(W)::value;
+        const uint64_t dx = d_x0 + ((w * C::X_BYTES) >> 4);
+        const uint32_t z_col = tm + C::COL_Z + w * 128;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          tc_mma_ts_w(z_col + 64, z_col + 8 * kk, dx + ((kk * 2048) >> 4), ID_YD, kk > 0);
+        tc_commit_w(bar(YD_DONE0 + w));
+        tc_commit_w(bar(XEMPTY0 + w));
+      };
+      using I0 = std::integral_constant<uint32_t, 0>;
+      using I1 = std::integral_constant<uint32_t, 1>;
       uint32_t nds = 0, nyo = 0, ncb = 0, nyd = 0, nbc = 0;
       uint64_t t_last = 0;
       uint32_t idle = 0;
@@ -428,70 +490,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool did = false;
         // N <= 128: dS goes to a fresh buffer the state warps have read out;
         // N = 256: it accumulates onto the state the state warps decayed (HB_READY)
-        const bool ds_slot_ok =
-            NT == 1 ? (nds < (uint32_t)C::DSB ||
-                       tst(DS_FREE0 + nds % C::DSB, ((nds - C::DSB) / C::DSB) & 1))
-                    : tst(HB_READY0, nds & 1);
         if (nds < ntiles && tst(XW_READY0 + (nds & 1), (nds >> 1) & 1) &&
-            tst(BCFULL0 + nds % C::BS, (nds / C::BS) & 1) && ds_slot_ok) {
-          // dS = B_j^T XW : K = tokens; A = the B tile read MN-major (n), B = XW (p)
+            tst(BCFULL0 + nds % C::BS, (nds / C::BS) & 1) &&
+            (NT == 1 ? (nds < (uint32_t)C::DSB ||
+                        tst(DS_FREE0 + nds % C::DSB, ((nds - C::DSB) / C::DSB) & 1))
+                     : tst(HB_READY0, nds & 1))) {
           tc_fence_after();
-          const uint32_t w = nds & 1;
-          const uint64_t dbm = sdesc(bc_of(nds), kPanel, 1024);
-          const uint64_t dxw = sdesc(sbase + C::OFF_XW + w * kPanel, kPanel, 1024);
-          const uint32_t dcol = tmem + C::COL_DS + (nds % C::DSB) * NT * kPT;
-#pragma unroll
-          for (int mt = 0; mt < NT; ++mt)
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk)
-              tc_mma_w(dcol + mt * kPT, dbm + ((2 * mt * kPanel + kk * 2048) >> 4),
-                     dxw + ((kk * 2048) >> 4), ID_ST, NT == 2 || kk > 0);
-          tc_commit_w(bar(DS_DONE0 + w));
+          if (nds & 1) issue_ds(I1{}); else issue_ds(I0{});
           ++nds;
           did = true;
         } else if (nyo < ntiles && tst(HB_READY0 + nyo % C::HBS, (nyo / C::HBS) & 1) &&
                    tst(BCFULL0 + nyo % C::BS, (nyo / C::BS) & 1) &&
                    (nyo < 2 || tst(ZFREE0 + (nyo & 1), ((nyo - 2) >> 1) & 1))) {
-          // Yoff = C_j Hb_j : K = state dim; Hb rows are n (K), 128 bytes of p (MN)
           tc_fence_after();
-          const uint32_t w = nyo & 1;
-          const uint64_t dc = sdesc(bc_of(nyo) + C::BC1_BYTES, 16, 1024);
-          const uint64_t dhb = sdesc(sbase + C::OFF_HB + (nyo % C::HBS) * C::HB_BYTES, C::HB_BYTES, 1024);
-#pragma unroll
-          for (int kk = 0; kk < C::NPAD / 16; ++kk)
-            tc_mma_w(tmem + C::COL_YO + w * kPT, dc + (((kk >> 2) * kPanel + (kk & 3) * 32) >> 4),
-                   dhb + ((kk * 2048) >> 4), ID_YOFF, kk > 0);
-          tc_commit_w(bar(YO_DONE0 + w));
+          if (nyo & 1) issue_yo(I1{}); else issue_yo(I0{});
           ++nyo;
           did = true;
         } else if (ncb < ntiles && tst(BCFULL0 + ncb % C::BS, (ncb / C::BS) & 1) &&
                    (ncb < 2 || tst(ZFREE0 + (ncb & 1), ((ncb - 2) >> 1) & 1))) {
-          // Z[w] = C_j B_j^T : K = state dim
           tc_fence_after();
-          const uint32_t w = ncb & 1;
-          const uint64_t dc = sdesc(bc_of(ncb) + C::BC1_BYTES, 16, 1024);
-          const uint64_t db = sdesc(bc_of(ncb), 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < C::NPAD / 16; ++kk) {
-            const uint64_t off = ((kk >> 2) * kPanel + (kk & 3) * 32) >> 4;
-            tc_mma_w(tmem + C::COL_Z + w * 128, dc + off, db + off, ID_CB, kk > 0);
-          }
-          tc_commit_w(bar(CB_DONE0 + w));
+          if (ncb & 1) issue_cb(I1{}); else issue_cb(I0{});
           ++ncb;
           did = true;
         } else if (nyd < ncb && tst(M_READY0 + (nyd & 1), (nyd >> 1) & 1) &&
                    tst(XFULL0 + nyd % C::XS, (nyd / C::XS) & 1)) {
-          // Ydiag = M X_j : K = tokens.  M sits in TMEM as bf16 pairs (the 16 tokens
-          // of K step kk in columns 8kk..8kk+7 of the Z buffer); Ydiag goes next to it
           tc_fence_after();
-          const uint32_t w = nyd & 1;
-          const uint64_t dx = sdesc(sbase + C::OFF_X + (nyd % C::XS) * C::X_BYTES, kPanel, 1024);
-          const uint32_t z_col = tmem + C::COL_Z + w * 128;
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            tc_mma_ts_w(z_col + 64, z_col + 8 * kk, dx + ((kk * 2048) >> 4), ID_YD, kk > 0);
-          tc_commit_w(bar(YD_DONE0 + w));
-          tc_commit_w(bar(XEMPTY0 + nyd % C::XS));
+          if (nyd & 1) issue_yd(I1{}); else issue_yd(I0{});
           ++nyd;
           did = true;
         }
@@ -516,8 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // every product this thread issued has completed once TEARDOWN fires; bounded
-      // by time only, since TMEM is freed below
+      // every product this warp issued has completed once TEARDOWN fires; bounded by
+      // time only, since TMEM is freed below
       tc_commit_w(bar(TEARDOWN));
       if (!wait_drain(bar(TEARDOWN), 0, 2000000000ull)) set_status(kp.status, SSD_ERR_TIMEOUT);
     }

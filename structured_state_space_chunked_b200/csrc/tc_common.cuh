@@ -135,6 +135,16 @@ __device__ __forceinline__ void tma_3d_w(uint32_t dst, const CUtensorMap* m, uin
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// L2 prefetch of a 2-D tensor tile (no shared memory, no barrier), issued by lane 0
+// of a warp-wide call
+__device__ __forceinline__ void tma_prefetch_2d_w(const CUtensorMap* m, int c0, int c1) {
+  asm volatile(
+      "{\n .reg .pred e;\n .reg .u32 l;\n mov.u32 l, %%laneid;\n setp.eq.u32 e, l, 0;\n"
+      " @e cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];\n}\n" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(c0), "r"(c1)
+      : "memory");
+}
 __device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
