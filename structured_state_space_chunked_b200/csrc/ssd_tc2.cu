@@ -27,10 +27,10 @@
 // the decomposition uses between chunks (the mask restricted to a strictly lower
 // block is rank one, §3.2.2), equal to the quadratic form up to rounding.
 //
-// Warps: 0-3 the state chain (S), 4-7 and 8-11 two epilogue groups taking
-// alternate tiles (cumulative decay, w o x, the decay mask written over C B^T in
-// TMEM as bf16, the outputs), 12 the MMA issuer and TMEM owner, 13 the TMA
-// producer.  The issuer and producer warps run their loops with all 32 lanes and
+// Warps: 0-3 the state chain (S; also w o x, the B operand of dS), 4-7 and 8-11
+// two epilogue groups taking alternate tiles (cumulative decay, the decay mask
+// written over C B^T in TMEM as bf16, the outputs), 12 the MMA issuer and TMEM
+// owner, 13 the TMA producer.  The issuer and producer warps run their loops with all 32 lanes and
 // warp-uniform state; an elect.sync inside each instruction's asm block picks the
 // lane that issues it, so descriptors and coordinates stay in uniform registers.  Every mbarrier wait is bounded; a wait that runs out records
 // SSD_ERR_TIMEOUT in the status word, raises the CTA's abort flag and every role
@@ -90,17 +90,18 @@ static_assert(Cfg2<1>::COL_DS + Cfg2<1>::DSB * 64 <= 512, "tmem budget");
 static_assert(Cfg2<2>::COL_DS + 2 * 64 <= 512, "tmem budget");
 
 enum Bar2 {
-  XFULL0 = 0, XFULL1, XEMPTY0, XEMPTY1,   // x tile slots (TMA -> readers; Ydiag commit -> TMA)
+  XFULL0 = 0, XFULL1, XEMPTY0, XEMPTY1,   // x tile slots (TMA -> readers; MMA commit -> TMA)
   BCFULL0, BCFULL1, BCEMPTY0, BCEMPTY1,   // B/C tile slots (TMA -> MMA; MMA commit -> TMA)
   CB_DONE0, CB_DONE1,     // C B^T in the group's Z buffer (MMA -> epilogue group)
   M_READY0, M_READY1,     // mask written over it (group -> MMA)
   YD_DONE0, YD_DONE1,     // Ydiag done (MMA -> group)
-  XW_READY0, XW_READY1,   // w o x written (group -> MMA)
+  XW_READY0, XW_READY1,   // w o x written (state warps -> MMA)
   DS_DONE0, DS_DONE1,     // dS of the group's tile done (MMA -> state warps and the group)
   YO_DONE0, YO_DONE1,     // left factors done (MMA -> group and state warps)
   ZFREE0, ZFREE1,         // the group read Ydiag and Yoff (group -> MMA)
   HB_READY0, HB_READY1,   // bf16 state copy written (state warps -> MMA), per slot
   DS_FREE0, DS_FREE1,     // dS buffer read (state warps -> MMA), per buffer
+  XWBUF_FREE0, XWBUF_FREE1, // the group copied out y staged in its w o x buffer (group -> state warps)
   STALL,                  // nothing arrives here: the forced-timeout test waits on it
   TEARDOWN, NBAR
 };
@@ -349,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < NBAR; ++i) {
       const bool group = i == M_READY0 || i == M_READY1 || i == XW_READY0 || i == XW_READY1 ||
                          i == ZFREE0 || i == ZFREE1 || i == HB_READY0 || i == HB_READY1 ||
-                         i == DS_FREE0 || i == DS_FREE1;
+                         i == DS_FREE0 || i == DS_FREE1 || i == XWBUF_FREE0 || i == XWBUF_FREE1;
       mbar_init(bar(i), group ? 128 : 1);
     }
     fence_barrier_init();
@@ -479,11 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kTile / 16; ++kk)
           tc_mma_ts_w(z_col + 64, z_col + 8 * kk, dx + ((kk * 2048) >> 4), ID_YD, kk > 0);
         tc_commit_w(bar(YD_DONE0 + w));
-        tc_commit_w(bar(XEMPTY0 + w));
       };
       using I0 = std::integral_constant<uint32_t, 0>;
       using I1 = std::integral_constant<uint32_t, 1>;
-      uint32_t nds = 0, nyo = 0, ncb = 0, nyd = 0, nbc = 0;
+      uint32_t nds = 0, nyo = 0, ncb = 0, nyd = 0, nbc = 0, nxe = 0;
       uint64_t t_last = 0;
       uint32_t idle = 0;
       while (nyd < ntiles || nds < ntiles || nyo < ntiles) {
@@ -523,6 +523,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit_w(bar(BCEMPTY0 + nbc % C::BS));
           ++nbc;
         }
+        // an x slot is free once Ydiag read it and the state warps built w o x from it
+        // (dS of the tile is issued only after that)
+        while (nxe < nyd && nxe < nds) {
+          tc_commit_w(bar(XEMPTY0 + nxe % C::XS));
+          ++nxe;
+        }
         if (did) {
           idle = 0;
           t_last = 0;
@@ -552,6 +558,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3, r = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     float* ws = ws_all + 8;  // two 4-float halves, alternating by tile
+    // XW = w o x_j, the MN-major B operand of dS_j, w_r = exp(cs_last - cs_r) delta_r,
+    // written into the w o x buffer of the tile's parity once the epilogue group has
+    // copied out the y tile it staged there two tiles earlier
+    auto make_xw = [&](uint32_t j, const Scan& sc, bool ok) -> bool {
+      const uint32_t wb = j & 1;
+      if (ok && j >= 2) ok = __all_sync(0xffffffffu, waitb(XWBUF_FREE0 + wb, ((j - 2) >> 1) & 1));
+      if (ok) ok = __all_sync(0xffffffffu, waitb(XFULL0 + j % C::XS, (j / C::XS) & 1));
+      if (ok) {
+        const float wr = ex2(sc.e3 - sc.cs) * sc.dl;
+        const uint32_t xrow = sbase + C::OFF_X + (j % C::XS) * C::X_BYTES;
+        const uint32_t xw_base = sbase + C::OFF_XW + wb * kPanel;
+#pragma unroll
+        for (int cidx = 0; cidx < 8; ++cidx) {
+          const uint4 xv = ld_shared_v4(xrow + swz((uint32_t)r, (uint32_t)cidx));
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+          const float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
+          const float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
+          st_shared_v4(xw_base + swz((uint32_t)r, (uint32_t)cidx), pack_bf16(wr * f0.x, wr * f0.y),
+                       pack_bf16(wr * f1.x, wr * f1.y), pack_bf16(wr * f2.x, wr * f2.y),
+                       pack_bf16(wr * f3.x, wr * f3.y));
+        }
+        fence_async_smem();
+        mbar_arrive(bar(XW_READY0 + wb));
+      }
+      return ok;
+    };
     // documents without tokens: their final state is their initial state (or zero)
     if (kp.final_states) {
       for (int u = blockIdx.x; u < kp.units; u += gridDim.x) {
@@ -632,6 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(bar(HB_READY0));
         }
+        ok = make_xw(j, sc, ok);
         // the unit's last tile: the final state once its update is done
         if (ok && cur.jt == U.ntiles - 1) {
           ok = __all_sync(0xffffffffu, waitb(DS_DONE0 + (j & 1), (j >> 1) & 1));
@@ -702,6 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_async_smem();
         mbar_arrive(bar(HB_READY0 + j % C::HBS));
       }
+      ok = make_xw(j, sc, ok);
       // S <- exp(cs_last) S + dS_j
       if (ok) ok = __all_sync(0xffffffffu, waitb(DS_DONE0 + (j & 1), (j >> 1) & 1));
       if (ok) {
@@ -770,8 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float cs_end = q == 0 ? sc.e0 : q == 1 ? sc.e1 : q == 2 ? sc.e2 : sc.e3;
         vw[r] = ex2(cs_end - sc.cs) * sc.dl;
       }
-      const float wr = ex2(sc.e3 - sc.cs) * sc.dl;  // exp(cs_last - cs) delta
-      const float el = ex2(sc.cs);                  // exp(cs)
+      const float el = ex2(sc.cs);  // exp(cs)
       Cursor nxt = cur;
       cursor_next(kp, nxt);
       cursor_next(kp, nxt);
@@ -779,26 +812,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = group_and(gid, ok);  // vw visible to the group
       if (!ok) break;
 
-      // ---- E4: XW = w o x_j (MN-major B operand of dS) ----
-      ok = __all_sync(0xffffffffu, waitb(XFULL0 + j % C::XS, (j / C::XS) & 1));
-      if (ok) {
-        const uint32_t xrow = sbase + C::OFF_X + (j % C::XS) * C::X_BYTES;
-#pragma unroll
-        for (int cidx = 0; cidx < 8; ++cidx) {
-          const uint4 xv = ld_shared_v4(xrow + swz((uint32_t)r, (uint32_t)cidx));
-          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
-          const float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
-          const float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
-          st_shared_v4(xw_base + swz((uint32_t)r, (uint32_t)cidx), pack_bf16(wr * f0.x, wr * f0.y),
-                       pack_bf16(wr * f1.x, wr * f1.y), pack_bf16(wr * f2.x, wr * f2.y),
-                       pack_bf16(wr * f3.x, wr * f3.y));
-        }
-        fence_async_smem();
-        mbar_arrive(bar(XW_READY0 + w));
-      }
-
       // ---- E2: decay mask of the diagonal block, over C B^T in TMEM ----
-      if (ok) ok = __all_sync(0xffffffffu, waitb(CB_DONE0 + w, k & 1));
+      ok = __all_sync(0xffffffffu, waitb(CB_DONE0 + w, k & 1));
       if (ok) {
         tc_fence_after();
         if (q > 0) mask_off(zaddr, 0, sc.cs, sc.e0, vw);
@@ -840,8 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       {
         // 16-byte chunk e of the 128 x 128-byte tile: row e/8, chunk e%8; a warp
-        // instruction covers four whole rows.  The staging tile is next written by
-        // this group's next tile after the barriers of its E1.
+        // instruction covers four whole rows.
         __nv_bfloat16* ybase = kp.y + (int64_t)U.h * g.P + U.ps * kPT;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -851,6 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(ybase + (t0 + row) * (int64_t)g.H * g.P + c * 8) = v;
           }
         }
+        mbar_arrive(bar(XWBUF_FREE0 + w));  // the buffer takes w o x of tile j + 2
       }
       cur = nxt;
     }
