@@ -87,13 +87,15 @@ enum {
    * SSD_ERR_UNSUPPORTED.  Both widths compute the same result. */
   SSD_OPT_TC_UNIT_COLUMNS = 2,
   /* value: 1 .. 60,000,000 microseconds (default 2,000,000), the bound of every
-   * device-side wait of the tensor-core forward kernel on N <= 128.  A wait that
-   * runs out records SSD_ERR_TIMEOUT in the status word (ssd_get_status) and the
-   * kernel unwinds, leaving the outputs of that call undefined and the handle and
-   * context usable. */
+   * device-side wait of the tensor-core forward.  A value other than the default
+   * selects the tensor-core kernel with the register-resident state chain for every
+   * N <= 256 (it is the default kernel for N > 128; the one for N <= 128 bounds its
+   * waits at the default).  A wait that runs out records SSD_ERR_TIMEOUT in the
+   * status word (ssd_get_status) and the kernel unwinds, leaving the outputs of
+   * that call undefined and the handle and context usable. */
   SSD_OPT_WAIT_LIMIT_US = 3,
   /* value: 0 (default) or 1.  Failure-path test: with 1, every following
-   * ssd_forward on the tensor-core path (N <= 128, 64-column units) first waits on
+   * ssd_forward on the tensor-core path (64-column units) first waits on
    * a device barrier that nothing completes, so that wait runs out after the
    * SSD_OPT_WAIT_LIMIT_US bound and the call reports SSD_ERR_TIMEOUT through the
    * status word.  No GPU fault is involved.  Set it back to 0 to compute again. */

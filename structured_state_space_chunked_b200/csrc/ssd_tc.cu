@@ -802,7 +802,10 @@ size_t tc_workspace_bytes(const Geom&) { return 256; }
 cudaError_t tc_forward(const Geom& g, const Args& a, void*, int* status, cudaStream_t stream,
                        int num_sms, const TcOpts& opts) {
   if (opts.unit_columns == 128) return tc_wide_forward(g, a, status, stream, num_sms);
-  if (tc2_supported(g)) return tc2_forward(g, a, status, stream, num_sms, opts.wait_ns, opts.stall);
+  // N > 128, and any shape whose wait bound or forced-timeout test is set: the kernel
+  // of ssd_tc2.cu (its bounded waits take the handle's limit)
+  if (tc2_supported(g) || opts.stall || opts.wait_ns != TcOpts().wait_ns)
+    return tc2_forward(g, a, status, stream, num_sms, opts.wait_ns, opts.stall);
   CUtensorMap tx, tb, tc;
   const cuuint64_t T = (cuuint64_t)g.tokens;
   {

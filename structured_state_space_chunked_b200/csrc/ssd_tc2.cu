@@ -885,8 +885,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-// Shapes this kernel takes: those of the 64-column tensor-core path.
-bool tc2_supported(const Geom& g) { return g.N <= 256; }
+// Shapes this kernel takes: the 64-column tensor-core path with N > 128 (two lane
+// tiles of state).  For N <= 128 the kernel of ssd_tc.cu measured faster on every
+// benchmark shape, so it keeps those (this kernel computes them as well).
+bool tc2_supported(const Geom& g) { return g.N > 128 && g.N <= 256; }
 
 cudaError_t tc2_forward(const Geom& g, const Args& a, int* status, cudaStream_t stream, int num_sms,
                         unsigned long long wait_ns, int stall) {
