@@ -615,8 +615,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         Cursor nxt = cur;
         cursor_next(kp, nxt);
         pre = prefetch(kp, nxt, r);
+        // w o x of this tile first: it needs only x and the scan, and dS of the tile
+        // (which frees the B/C slot) waits for it
+        ok = make_xw(j, sc, ok);
         // the state after tile j-1 is complete, and its left factors read the bf16 copy
-        if (cur.jt > 0)
+        if (ok && cur.jt > 0)
           ok = __all_sync(0xffffffffu, waitb(DS_DONE0 + ((j - 1) & 1), ((j - 1) >> 1) & 1));
         if (ok && j > 0)
           ok = __all_sync(0xffffffffu, waitb(YO_DONE0 + ((j - 1) & 1), ((j - 1) >> 1) & 1));
@@ -664,7 +667,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(bar(HB_READY0));
         }
-        ok = make_xw(j, sc, ok);
         // the unit's last tile: the final state once its update is done
         if (ok && cur.jt == U.ntiles - 1) {
           ok = __all_sync(0xffffffffu, waitb(DS_DONE0 + (j & 1), (j >> 1) & 1));
