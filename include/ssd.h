@@ -66,7 +66,10 @@ enum {
   SSD_ERR_TIMEOUT = -4,     /* a device-side bounded wait gave up (status word) */
   SSD_ERR_OOM = -5,         /* device allocation failed */
   SSD_ERR_BAD_SEQLENS = -6, /* cu_seqlens not 0 = c[0] <= ... <= c[n] = tokens (status word) */
-  SSD_ERR_SCRATCH_TOO_SMALL = -7 /* ssd_forward_noalloc: problem needs more than its fixed scratch */
+  SSD_ERR_SCRATCH_TOO_SMALL = -7, /* ssd_forward_noalloc: problem needs more than its fixed scratch */
+  SSD_ERR_DEBUG_CHECK = -8  /* debug builds only (SSD_DEBUG): a device-side bounds or barrier-phase
+                             * check failed (status word; the offending source line is in the
+                             * word after it) */
 };
 
 /* kernel paths (ssd_plan_t.path, SSD_OPT_FORCE_PATH) */
@@ -404,6 +407,14 @@ SSD_API int ssd_forward_noalloc(const ssd_desc_t* desc, const void* x, const voi
                                 const float* dt_bias, int chunk_size, const float* initial_states,
                                 const int32_t* cu_seqlens, int num_docs, void* y,
                                 float* final_states, int* status, ssd_stream_t stream);
+
+/* Debug builds: the source line of the first failed device-side check recorded in
+ * the handle's status word since the handle was created (0: none).  Synchronises
+ * the device.  Release builds record nothing and return 0. */
+SSD_API int ssd_debug_line(ssd_handle_t h);
+
+/* 1 for a library built with device-side checks (`build.py --debug`), 0 otherwise. */
+SSD_API int ssd_debug_build(void);
 
 /* Static string naming a return code. */
 SSD_API const char* ssd_error_string(int code);

@@ -1,9 +1,11 @@
 """Build libssd_b200.so (the CUDA library behind include/ssd.h) for sm_100a.
 
-    python -m structured_state_space_chunked_b200.build
+    python -m structured_state_space_chunked_b200.build [--force] [--debug]
 
 compiles every ``csrc/*.cu`` with nvcc into one shared library in this package
-directory.  The library links the CUDA runtime statically and the driver API is
+directory.  ``--debug`` builds ``libssd_b200_debug.so`` instead, with -DSSD_DEBUG:
+device-side bounds and barrier-phase checks that report SSD_ERR_DEBUG_CHECK through
+the status word (the binding loads it when SSD_B200_LIBRARY names it).  The library links the CUDA runtime statically and the driver API is
 reached through ``cudaGetDriverEntryPoint``, so loading it needs no GPU.
 """
 
@@ -19,6 +21,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libssd_b200.so")
+DEBUG_LIB = os.path.join(PKG, "libssd_b200_debug.so")
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
@@ -44,43 +47,45 @@ def headers():
     return sorted(glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in sources() + headers())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
     objs = []
-    build_dir = os.path.join(PKG, "_build")
+    build_dir = os.path.join(PKG, "_build_debug" if debug else "_build")
     os.makedirs(build_dir, exist_ok=True)
     logs = []
     for src in sources():
         obj = os.path.join(build_dir, os.path.basename(src) + ".o")
-        cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
+        cmd = [nvcc(), *NVCC_FLAGS, *(["-DSSD_DEBUG"] if debug else []), "-I",
+               os.path.join(ROOT, "include"), "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         logs.append(r.stdout + r.stderr)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError(f"nvcc failed on {src}")
         objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs,
            "-Xcompiler", "-fPIC"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("nvcc link failed")
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
     with open(os.path.join(build_dir, "ptxas.log"), "w") as f:
         f.write("\n".join(logs))
     if verbose:
         print("\n".join(logs))
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -188,6 +188,7 @@ int ssd_forward(ssd_handle_t h, const void* x, const void* dt, const float* A, c
                 const void* C, const float* D, const float* dt_bias, int chunk_size,
                 const float* initial_states, const int32_t* cu_seqlens, int num_docs, void* y,
                 float* final_states, ssd_stream_t stream_) {
+  ssd::NvtxRange nvtx_range("ssd_forward");
   if (!h) return SSD_ERR_INVALID_ARG;
   const ssd_desc_t& d = h->desc;
   int rc = check_call(d, chunk_size, cu_seqlens, num_docs);
@@ -243,6 +244,7 @@ int ssd_backward(ssd_handle_t h, const void* x, const void* dt, const float* A, 
                  const int32_t* cu_seqlens, int num_docs, const void* dy, const float* dfinal_states,
                  float* dx, float* ddt, float* dA, float* dB, float* dC, float* dD, float* ddt_bias,
                  float* dinitial_states, ssd_stream_t stream_) {
+  ssd::NvtxRange nvtx_range("ssd_backward");
   if (!h) return SSD_ERR_INVALID_ARG;
   const ssd_desc_t& d = h->desc;
   int rc = check_call(d, ssd::kBwdQ, cu_seqlens, num_docs);
@@ -295,6 +297,7 @@ int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* 
                     const void* C, const float* D, const float* dt_bias, int chunk_size,
                     const int32_t* cu_seqlens, int num_docs, int feature_map, int normalize, void* y,
                     float* final_states, ssd_stream_t stream_) {
+  ssd::NvtxRange nvtx_range("ssd_forward_ext");
   if (!h) return SSD_ERR_INVALID_ARG;
   const ssd_desc_t& d = h->desc;
   int rc = check_call(d, chunk_size, cu_seqlens, num_docs);
@@ -382,6 +385,7 @@ int ssd_forward_host(ssd_handle_t h, const void* x, const void* dt, const float*
                      const void* B, const void* C, const float* D, const float* dt_bias,
                      int chunk_size, const float* initial_states, const int32_t* cu_seqlens,
                      int num_docs, void* y, float* final_states, ssd_stream_t stream_) {
+  ssd::NvtxRange nvtx_range("ssd_forward_host");
   if (!h) return SSD_ERR_INVALID_ARG;
   const ssd_desc_t& d = h->desc;
   int rc = check_call(d, chunk_size, cu_seqlens, num_docs);
@@ -470,6 +474,20 @@ int ssd_get_status(ssd_handle_t h, ssd_stream_t stream_) {
   return v;
 }
 
+int ssd_debug_line(ssd_handle_t h) {
+  if (!h) return SSD_ERR_INVALID_ARG;
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess) return SSD_ERR_CUDA;
+  int v = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&v, h->status + 1, sizeof(int), cudaMemcpyDeviceToHost);
+  if (cur != h->device) cudaSetDevice(cur);
+  return e == cudaSuccess ? v : SSD_ERR_CUDA;
+}
+
+int ssd_debug_build(void) { return SSD_DEBUG_ON; }
+
 int ssd_destroy(ssd_handle_t h) {
   if (!h) return SSD_OK;
   int cur = 0;
@@ -496,6 +514,8 @@ const char* ssd_error_string(int code) {
     case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: a device-side wait gave up";
     case SSD_ERR_OOM: return "SSD_ERR_OOM: device allocation failed";
     case SSD_ERR_BAD_SEQLENS: return "SSD_ERR_BAD_SEQLENS: cu_seqlens is not a valid partition";
+    case SSD_ERR_DEBUG_CHECK:
+      return "SSD_ERR_DEBUG_CHECK: a device-side bounds or barrier-phase check failed (debug build)";
     case SSD_ERR_SCRATCH_TOO_SMALL:
       return "SSD_ERR_SCRATCH_TOO_SMALL: the problem needs more scratch than the fixed array";
     default: return "SSD_ERR_UNKNOWN";

@@ -7,6 +7,8 @@
 
 #include "../../include/ssd.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace ssd {
 
 // Problem geometry of one ssd_forward call, passed by value to kernels.
@@ -36,10 +38,37 @@ struct Args {
   float* final_states;
 };
 
+// An NVTX range around the launches of one entry point (visible in Nsight timelines;
+// without a profiling tool attached a push/pop costs a few nanoseconds).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Device status word values are the negative SSD_ERR_* codes; 0 = ok.
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
+
+// Debug builds (-DSSD_DEBUG, `build.py --debug`): device-side checks of indices and
+// barrier phases.  A failed check records SSD_ERR_DEBUG_CHECK in the status word and
+// the source line in the word after it, and the access it guards is skipped where the
+// call site says so; it never traps.  Release builds compile the checks away.
+#ifdef SSD_DEBUG
+#define SSD_DEBUG_ON 1
+__device__ __forceinline__ bool debug_check(bool ok, int* status, int line) {
+  if (!ok && status) {
+    if (atomicCAS(status, 0, SSD_ERR_DEBUG_CHECK) == 0) status[1] = line;
+  }
+  return ok;
+}
+#define SSD_CHECK(cond, status) ::ssd::debug_check((cond), (status), __LINE__)
+#else
+#define SSD_DEBUG_ON 0
+#define SSD_CHECK(cond, status) true
+#endif
 
 __device__ __forceinline__ float load_f(const void* p, int64_t i, int bf16) {
   return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i])

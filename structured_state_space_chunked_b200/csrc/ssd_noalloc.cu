@@ -62,6 +62,7 @@ extern "C" SSD_API int ssd_forward_noalloc(const ssd_desc_t* desc, const void* x
                                            const int32_t* cu_seqlens, int num_docs, void* y,
                                            float* final_states, int* status,
                                            ssd_stream_t stream_) {
+  ssd::NvtxRange nvtx_range("ssd_forward_noalloc");
   int rc = ssd_validate_desc(desc);
   if (rc) return rc;
   const ssd_desc_t& d = *desc;

@@ -94,6 +94,7 @@ bool aligned(const void* q, size_t a) { return ((uintptr_t)q % a) == 0; }
 extern "C" SSD_API int ssd_step(const ssd_desc_t* desc, const void* x, const void* dt,
                                 const float* A, const void* B, const void* C, const float* D,
                                 const float* dt_bias, float* state, void* y, ssd_stream_t stream) {
+  ssd::NvtxRange nvtx_range("ssd_step");
   using ssd::aligned;
   if (!desc) return SSD_ERR_INVALID_ARG;
   const ssd_desc_t& d = *desc;

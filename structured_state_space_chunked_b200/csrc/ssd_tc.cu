@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = bar(FULL0 + s);
         const int g_idx = c.U.h / (g.H / g.G);
         const int t0 = (int)(c.U.start + (int64_t)c.jt * kTile);
+        SSD_CHECK(t0 >= 0 && t0 < g.tokens && g_idx < g.G && (c.U.ps + 1) * kPT <= g.P, kp.status);
         mbar_expect_tx(fb, C::TX_BYTES);
         tma_2d(st, &tm_x, fb, c.U.h * g.P + c.U.ps * kPT, t0);
 #pragma unroll
@@ -716,7 +717,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int e = tid + 128 * i, row = e >> 3, c = e & 7;
-          if (row < len) {
+          if (row < len && SSD_CHECK(t0 + row < g.tokens && U.h * g.P + U.ps * kPT + c * 8 + 8 <= g.H * g.P,
+                                     kp.status)) {
             const uint4 v = ld_shared_v4(xw_base + swz((uint32_t)row, (uint32_t)c));
             *reinterpret_cast<uint4*>(ybase + (t0 + row) * (int64_t)g.H * g.P + c * 8) = v;
           }

@@ -316,6 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* ws_all = reinterpret_cast<float*>(smem + C::OFF_WS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS);
   int* bad_flag = reinterpret_cast<int*>(smem + C::OFF_FLAGS + 4);
+  // debug builds: fills of each x and B/C slot (TMA producer) and products issued
+  // (MMA issuer), read by the barrier-phase checks
+  volatile int* dbg = reinterpret_cast<volatile int*>(smem + C::OFF_FLAGS + 8);
+  enum { DBG_XFILL = 0, DBG_BFILL = 2, DBG_NCB = 4, DBG_NDS = 5, DBG_N = 6 };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_TMEM);
   auto bar = [&](int i) { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
   const Geom& g = kp.g;
@@ -328,6 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     *bad_flag = (sbase & 1023u) != 0 ? 2 : 0;
+    for (int i = 0; i < DBG_N; ++i) dbg[i] = 0;
   }
   __syncthreads();
   if (g.varlen) {
@@ -379,6 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const uint32_t s = nx % C::XS;
         if (nx >= C::XS && !__all_sync(0xffffffffu, waitb(XEMPTY0 + s, ((nx - C::XS) / C::XS) & 1))) break;
+        if (SSD_DEBUG_ON) {
+          SSD_CHECK(t0 >= 0 && t0 < g.tokens && c.U.h < g.H && (c.U.ps + 1) * kPT <= g.P, kp.status);
+          if (lane == 0) dbg[DBG_XFILL + s] = (int)(nx / C::XS + 1);
+          __threadfence_block();
+        }
         mbar_expect_tx_w(bar(XFULL0 + s), C::X_BYTES);
         tma_2d_w(sbase + C::OFF_X + s * C::X_BYTES, &tm_x, bar(XFULL0 + s), c.U.h * g.P + c.U.ps * kPT, t0);
         ++nx;
@@ -388,6 +398,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (nbc >= C::BS && !__all_sync(0xffffffffu, waitb(BCEMPTY0 + s, ((nbc - C::BS) / C::BS) & 1))) break;
         const uint32_t st = sbase + C::OFF_BC + s * C::BC_BYTES;
         const int gi = c.U.h / (g.H / g.G);
+        if (SSD_DEBUG_ON) {
+          SSD_CHECK(gi >= 0 && gi < g.G, kp.status);
+          if (lane == 0) dbg[DBG_BFILL + s] = (int)(nbc / C::BS + 1);
+          __threadfence_block();
+        }
         mbar_expect_tx_w(bar(BCFULL0 + s), C::BC_BYTES);
 #pragma unroll
         for (int q = 0; q < C::NPANEL; ++q) {
@@ -496,8 +511,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tst(DS_FREE0 + nds % C::DSB, ((nds - C::DSB) / C::DSB) & 1))
                      : tst(HB_READY0, nds & 1))) {
           tc_fence_after();
+          SSD_CHECK(dbg[DBG_BFILL + nds % C::BS] == (int)(nds / C::BS + 1), kp.status);
           if (nds & 1) issue_ds(I1{}); else issue_ds(I0{});
           ++nds;
+          if (SSD_DEBUG_ON && lane == 0) dbg[DBG_NDS] = (int)nds;
           did = true;
         } else if (nyo < ntiles && tst(HB_READY0 + nyo % C::HBS, (nyo / C::HBS) & 1) &&
                    tst(BCFULL0 + nyo % C::BS, (nyo / C::BS) & 1) &&
@@ -509,12 +526,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (ncb < ntiles && tst(BCFULL0 + ncb % C::BS, (ncb / C::BS) & 1) &&
                    (ncb < 2 || tst(ZFREE0 + (ncb & 1), ((ncb - 2) >> 1) & 1))) {
           tc_fence_after();
+          // the B/C slot holds this tile's fill, not an earlier one
+          SSD_CHECK(dbg[DBG_BFILL + ncb % C::BS] == (int)(ncb / C::BS + 1), kp.status);
           if (ncb & 1) issue_cb(I1{}); else issue_cb(I0{});
           ++ncb;
+          if (SSD_DEBUG_ON && lane == 0) dbg[DBG_NCB] = (int)ncb;
           did = true;
         } else if (nyd < ncb && tst(M_READY0 + (nyd & 1), (nyd >> 1) & 1) &&
                    tst(XFULL0 + nyd % C::XS, (nyd / C::XS) & 1)) {
           tc_fence_after();
+          SSD_CHECK(dbg[DBG_XFILL + nyd % C::XS] == (int)(nyd / C::XS + 1), kp.status);
           if (nyd & 1) issue_yd(I1{}); else issue_yd(I0{});
           ++nyd;
           did = true;
@@ -670,6 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the unit's last tile: the final state once its update is done
         if (ok && cur.jt == U.ntiles - 1) {
           ok = __all_sync(0xffffffffu, waitb(DS_DONE0 + (j & 1), (j >> 1) & 1));
+          if (ok) SSD_CHECK(dbg[DBG_NDS] >= (int)(j + 1), kp.status);
           if (ok) {
             tc_fence_after();
 #pragma unroll 1
@@ -740,6 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = make_xw(j, sc, ok);
       // S <- exp(cs_last) S + dS_j
       if (ok) ok = __all_sync(0xffffffffu, waitb(DS_DONE0 + (j & 1), (j >> 1) & 1));
+      if (ok) SSD_CHECK(dbg[DBG_NDS] >= (int)(j + 1), kp.status);  // dS of this tile was issued
       if (ok) {
         tc_fence_after();
         const float decay = ex2(sc.e3);
@@ -817,6 +840,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- E2: decay mask of the diagonal block, over C B^T in TMEM ----
       ok = __all_sync(0xffffffffu, waitb(CB_DONE0 + w, k & 1));
       if (ok) {
+        SSD_CHECK(dbg[DBG_NCB] >= (int)(j + 1), kp.status);
         tc_fence_after();
         if (q > 0) mask_off(zaddr, 0, sc.cs, sc.e0, vw);
         if (q > 1) mask_off(zaddr, 1, sc.cs, sc.e1, vw);
@@ -862,7 +886,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int e = r + 128 * i, row = e >> 3, c = e & 7;
-          if (row < len) {
+          if (row < len && SSD_CHECK(t0 + row < g.tokens && U.h * g.P + U.ps * kPT + c * 8 + 8 <= g.H * g.P,
+                                     kp.status)) {
             const uint4 v = ld_shared_v4(xw_base + swz((uint32_t)row, (uint32_t)c));
             *reinterpret_cast<uint4*>(ybase + (t0 + row) * (int64_t)g.H * g.P + c * 8) = v;
           }

@@ -14,7 +14,10 @@ from typing import Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd_b200.so")
+# the library this binding loads: the in-package build, or the one SSD_B200_LIBRARY
+# names (e.g. libssd_b200_debug.so from `build.py --debug`)
+_LIB_PATH = os.environ.get("SSD_B200_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libssd_b200.so")
 _lib = None
 
 SSD_F32, SSD_BF16 = 0, 1
@@ -26,7 +29,7 @@ SSD_OPT_TEST_FORCE_TIMEOUT = 4
 ERRORS = {
     0: "SSD_OK", -1: "SSD_ERR_INVALID_ARG", -2: "SSD_ERR_UNSUPPORTED", -3: "SSD_ERR_CUDA",
     -4: "SSD_ERR_TIMEOUT", -5: "SSD_ERR_OOM", -6: "SSD_ERR_BAD_SEQLENS",
-    -7: "SSD_ERR_SCRATCH_TOO_SMALL",
+    -7: "SSD_ERR_SCRATCH_TOO_SMALL", -8: "SSD_ERR_DEBUG_CHECK",
 }
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -35,7 +38,7 @@ ABI_SYMBOLS = (
     "ssd_validate_desc", "ssd_plan", "ssd_create", "ssd_set_option", "ssd_forward",
     "ssd_forward_host", "ssd_get_status", "ssd_destroy", "ssd_error_string", "ssd_version",
     "ssd_forward_noalloc", "ssd_step", "ssd_cp_logdecay", "ssd_cp_combine", "ssd_cp_correct",
-    "ssd_backward", "ssd_feature_map_dim", "ssd_forward_ext",
+    "ssd_backward", "ssd_feature_map_dim", "ssd_forward_ext", "ssd_debug_line", "ssd_debug_build",
 )
 
 
@@ -99,6 +102,9 @@ def lib():
         for name in ("ssd_cp_logdecay", "ssd_cp_combine", "ssd_cp_correct"):
             getattr(L, name).restype = ctypes.c_int
         L.ssd_destroy.argtypes = [vp]
+        L.ssd_debug_line.argtypes = [vp]
+        L.ssd_debug_line.restype = ctypes.c_int
+        L.ssd_debug_build.restype = ctypes.c_int
         L.ssd_error_string.argtypes = [i32]
         L.ssd_error_string.restype = ctypes.c_char_p
         L.ssd_version.restype = ctypes.c_char_p
@@ -322,6 +328,11 @@ class SSD:
     def status(self, stream=None) -> int:
         """``ssd_get_status``: synchronise and return/clear the device status word."""
         return int(lib().ssd_get_status(self._h, _stream_ptr(stream)))
+
+    def debug_line(self) -> int:
+        """``ssd_debug_line``: source line of the first failed device-side check (debug
+        builds; 0 when none failed or in a release build)."""
+        return int(lib().ssd_debug_line(self._h))
 
     def close(self):
         if getattr(self, "_h", None):
