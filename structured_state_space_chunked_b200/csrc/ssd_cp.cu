@@ -28,62 +28,37 @@ namespace {
 constexpr int kScanThreads = 256;
 
 // cs[b, t, h] = sum_{k <= t} softplus(dt + dt_bias) A over the slice; ld[b, h] = cs at the
-// last token.  One CTA per (b, block of 32 heads).  The tokens go in tiles of 256: the
-// tile of delta A is loaded with consecutive threads on consecutive heads (the
-// contiguous dimension of dt and cs) into shared memory, each warp scans four heads
-// along the tokens (eight 32-token warp scans with a running carry), and the tile of
-// cs goes back with the same coalesced pattern.
-constexpr int kLdHeads = 32, kLdTok = 256, kLdPad = kLdTok + 1;
+// last token.  One CTA per (b, h), the tokens in blocks of 256 with a running carry.
 __global__ void __launch_bounds__(kScanThreads)
     cp_logdecay_kernel(int64_t L, int H, int in_bf16, const void* dt, const float* A,
                        const float* dt_bias, float* cs, float* ld) {
-  __shared__ float tile[kLdHeads * kLdPad];  // [head][token], padded against bank conflicts
-  const int b = blockIdx.x, h0 = blockIdx.y * kLdHeads;
+  __shared__ float warp_tot[kScanThreads / 32];
+  __shared__ float carry_s;
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int col = threadIdx.x % kLdHeads, h = h0 + col;  // the head this thread loads and stores
-  const float a = h < H ? A[h] : 0.f;
-  const float bias = (h < H && dt_bias) ? dt_bias[h] : 0.f;
-  float carry[kLdHeads / 8] = {0.f, 0.f, 0.f, 0.f};  // heads 4 wid .. 4 wid + 3
-  for (int64_t t0 = 0; t0 < L; t0 += kLdTok) {
-#pragma unroll 4
-    for (int i = 0; i < kLdTok * kLdHeads / kScanThreads; ++i) {
-      const int row = (i * kScanThreads + threadIdx.x) / kLdHeads;
-      const int64_t t = t0 + row;
-      float v = 0.f;
-      if (t < L && h < H) v = softplus_f(load_f(dt, ((int64_t)b * L + t) * H + h, in_bf16) + bias) * a;
-      tile[col * kLdPad + row] = v;
+  const float a = A[h], bias = dt_bias ? dt_bias[h] : 0.f;
+  if (threadIdx.x == 0) carry_s = 0.f;
+  __syncthreads();
+  for (int64_t t0 = 0; t0 < L; t0 += kScanThreads) {
+    const int64_t t = t0 + threadIdx.x;
+    float v = 0.f;
+    if (t < L) v = softplus_f(load_f(dt, ((int64_t)b * L + t) * H + h, in_bf16) + bias) * a;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
     }
+    if (lane == 31) warp_tot[wid] = v;
     __syncthreads();
-#pragma unroll
-    for (int c = 0; c < kLdHeads / 8; ++c) {
-      float* colp = tile + (4 * wid + c) * kLdPad;
-#pragma unroll
-      for (int k = 0; k < kLdTok / 32; ++k) {
-        float v = colp[32 * k + lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float u = __shfl_up_sync(0xffffffffu, v, o);
-          if (lane >= o) v += u;
-        }
-        v += carry[c];
-        colp[32 * k + lane] = v;
-        carry[c] = __shfl_sync(0xffffffffu, v, 31);
-      }
-    }
+    float base = carry_s;
+    for (int w = 0; w < wid; ++w) base += warp_tot[w];
+    v += base;
+    if (t < L) cs[((int64_t)b * L + t) * H + h] = v;
     __syncthreads();
-#pragma unroll 4
-    for (int i = 0; i < kLdTok * kLdHeads / kScanThreads; ++i) {
-      const int row = (i * kScanThreads + threadIdx.x) / kLdHeads;
-      const int64_t t = t0 + row;
-      if (t < L && h < H) cs[((int64_t)b * L + t) * H + h] = tile[col * kLdPad + row];
-    }
+    if (threadIdx.x == kScanThreads - 1) carry_s = v;  // inclusive sum at the block's end
     __syncthreads();
   }
-  if (lane == 0) {
-#pragma unroll
-    for (int c = 0; c < kLdHeads / 8; ++c)
-      if (h0 + 4 * wid + c < H) ld[(int64_t)b * H + h0 + 4 * wid + c] = carry[c];
-  }
+  if (threadIdx.x == 0) ld[bh] = carry_s;
 }
 
 // H_in and final state of rank r from every rank's local final state and log decay.
@@ -395,8 +370,8 @@ extern "C" SSD_API int ssd_cp_logdecay(const ssd_desc_t* desc, const void* dt, c
   const ssd_desc_t& d = *desc;
   if (d.batch == 0) return SSD_OK;
   if (!A || !cs || !logdecay || (d.seqlen > 0 && !dt)) return SSD_ERR_INVALID_ARG;
-  const dim3 grid((unsigned)d.batch, (unsigned)((d.nheads + ssd::kLdHeads - 1) / ssd::kLdHeads));
-  ssd::cp_logdecay_kernel<<<grid, ssd::kScanThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+  ssd::cp_logdecay_kernel<<<(unsigned)(d.batch * d.nheads), ssd::kScanThreads, 0,
+                            reinterpret_cast<cudaStream_t>(stream)>>>(
       d.seqlen, d.nheads, d.in_dtype == SSD_BF16, dt, A, dt_bias, cs, logdecay);
   return ssd::launch_rc();
 }

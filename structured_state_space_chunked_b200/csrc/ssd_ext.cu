@@ -185,6 +185,94 @@ __global__ void __launch_bounds__(32 * kDenWarps)
   }
 }
 
+// Steps (1) and (3) with the chunk's rows staged in shared memory: one CTA per
+// (chunk, block of 8 heads of one B/C group), one warp per head.  The chunk's B and C
+// rows (input dtype) and dt of the 8 heads are copied in once by the whole CTA
+// (consecutive threads on consecutive elements), so the serial token loop of each
+// warp reads shared memory only.  Same arithmetic, in the same order, as
+// den_chunk_kernel.
+constexpr int kDenHeads = 8;
+template <int E, bool OUT, typename TIn>
+__global__ void __launch_bounds__(32 * kDenHeads)
+    den_chunk_staged_kernel(Geom g, const int32_t* cu, SimtWorkspace ws, const void* dt,
+                            const float* A, const float* dt_bias, const void* B, const void* C,
+                            float* den) {
+  extern __shared__ __align__(16) unsigned char den_smem[];
+  TIn* sB = reinterpret_cast<TIn*>(den_smem);                 // [Q][N]
+  TIn* sC = sB + (size_t)kDenQ * g.N;                          // [Q][N]
+  float* sdt = reinterpret_cast<float*>(sC + (size_t)kDenQ * g.N);  // [Q][kDenHeads]
+  float (*part)[33] = reinterpret_cast<float (*)[33]>(sdt + kDenQ * kDenHeads);  // [8 warps * 32][33]
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t k = blockIdx.x;
+  const int h0 = blockIdx.y * kDenHeads, h = h0 + w, grp = h0 / (g.H / g.G), N = g.N;
+  ChunkInfo ci;
+  if (!chunk_info(g, cu, ws, k, &ci)) return;
+  // stage the chunk: B and C rows of the group, dt of the 8 heads
+  const int64_t row0 = (ci.start * g.G + grp) * (int64_t)N;
+  const int64_t rstride = (int64_t)g.G * N;
+  for (int i = threadIdx.x; i < ci.len * N; i += blockDim.x) {
+    const int t = i / N, n = i % N;
+    sB[i] = reinterpret_cast<const TIn*>(B)[row0 + t * rstride + n];
+    sC[i] = reinterpret_cast<const TIn*>(C)[row0 + t * rstride + n];
+  }
+  for (int i = threadIdx.x; i < ci.len * kDenHeads; i += blockDim.x) {
+    const int t = i / kDenHeads, hh = i % kDenHeads;
+    sdt[i] = load_f(dt, (ci.start + t) * g.H + h0 + hh, g.in_bf16);
+  }
+  __syncthreads();
+  const float a_h = A[h], bias = dt_bias ? dt_bias[h] : 0.f;
+  float* zs = ws.states + (k * g.H + h) * (int64_t)N;
+  float z[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int n = lane + 32 * e;
+    z[e] = (OUT && n < N) ? zs[n] : 0.f;
+  }
+  float cs = 0.f;
+  for (int tb = 0; tb < ci.len; tb += 32) {
+    const int nt = min(32, ci.len - tb);
+    for (int u = 0; u < nt; ++u) {
+      const int t = tb + u;
+      const float delta = softplus_f(sdt[t * kDenHeads + w] + bias);
+      const float decay = expf(delta * a_h);
+      cs = fmaf(delta, a_h, cs);
+      float sdot = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int n = lane + 32 * e;
+        if (n < N) {
+          z[e] = fmaf(decay, z[e], delta * (float)sB[t * N + n]);
+          if (OUT) sdot = fmaf((float)sC[t * N + n], z[e], sdot);
+        }
+      }
+      if (OUT) part[w * 32 + u][lane] = sdot;
+    }
+    if (OUT) {
+      __syncwarp();
+      if (lane < nt) {
+        float tot = 0.f;
+#pragma unroll 8
+        for (int q = 0; q < 32; ++q) tot += part[w * 32 + lane][q];
+        den[(ci.start + tb + lane) * g.H + h] = tot;
+      }
+      __syncwarp();
+    }
+  }
+  if (!OUT) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int n = lane + 32 * e;
+      if (n < N) zs[n] = z[e];
+    }
+    if (lane == 0) ws.cs[((int64_t)h * g.nchunks_max + k) * g.Q + g.Q - 1] = cs;
+  }
+}
+
+size_t den_staged_smem(const Geom& g) {
+  const size_t es = g.in_bf16 ? 2 : 4;
+  return 2 * (size_t)kDenQ * g.N * es + sizeof(float) * (kDenQ * kDenHeads + 32 * kDenHeads * 33);
+}
+
 // (2): per (document, head, state element), the chunks' end states become entering
 // states; eight chunks of loads are issued ahead of their dependent updates
 __global__ void __launch_bounds__(256) den_pass_kernel(Geom g, SimtWorkspace ws) {
@@ -275,6 +363,40 @@ cudaError_t den_scan(const Geom& g, const int32_t* cu, void* workspace, int* sta
   }
   const int64_t items = g.nchunks_max * g.H;
   if (items <= 0) return cudaSuccess;
+  const size_t sm = den_staged_smem(g);
+  if ((g.H / g.G) % kDenHeads == 0 && sm <= 227 * 1024) {
+    // chunk rows staged in shared memory (8 heads of a group per CTA)
+    const dim3 sgrid((unsigned)g.nchunks_max, (unsigned)(g.H / kDenHeads));
+    const int E = (g.N + 31) / 32;
+    cudaError_t e = cudaSuccess;
+    auto run = [&](auto kern) {
+      if (e != cudaSuccess) return;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if (e == cudaSuccess) {
+        kern<<<sgrid, 32 * kDenHeads, sm, stream>>>(g, cu, ws, dt, A, dt_bias, B, C, den);
+        e = cudaGetLastError();
+      }
+    };
+#define SSD_DEN_STAGED(EV, OUTV)                                                        \
+  (g.in_bf16 ? run(den_chunk_staged_kernel<EV, OUTV, __nv_bfloat16>)                     \
+             : run(den_chunk_staged_kernel<EV, OUTV, float>))
+#define SSD_DEN_SPICK(OUTV)                                \
+  if (E <= 1) SSD_DEN_STAGED(1, OUTV);                     \
+  else if (E <= 2) SSD_DEN_STAGED(2, OUTV);                \
+  else if (E <= 4) SSD_DEN_STAGED(4, OUTV);                \
+  else if (E <= 8) SSD_DEN_STAGED(8, OUTV);                \
+  else if (E <= 16) SSD_DEN_STAGED(16, OUTV);              \
+  else SSD_DEN_STAGED(32, OUTV)
+    SSD_DEN_SPICK(false);
+    if (e == cudaSuccess && g.ndocs > 0) {
+      den_pass_kernel<<<dim3(g.ndocs, g.H, (unsigned)((g.N + 255) / 256)), 256, 0, stream>>>(g, ws);
+      e = cudaGetLastError();
+    }
+    SSD_DEN_SPICK(true);
+#undef SSD_DEN_SPICK
+#undef SSD_DEN_STAGED
+    return e;
+  }
   const unsigned grid = (unsigned)((items + kDenWarps - 1) / kDenWarps);
   const int E = (g.N + 31) / 32;
 #define SSD_DEN_CASE(EV, OUTV)                                                                   \
