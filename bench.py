@@ -60,7 +60,7 @@ def algorithmic(w, ndocs):
 # the sources each measured kernel is built from (its recorded DRAM traffic stays
 # valid while these are unchanged)
 KERNEL_SOURCES = {
-    "tc": ("ssd_tc.cu", "tc_common.cuh", "ssd_internal.h"),
+    "tc": ("ssd_tc.cu", "ssd_tc2.cu", "tc_common.cuh", "ssd_internal.h"),
     "tc128": ("ssd_tc_wide.cu", "tc_common.cuh", "ssd_internal.h"),
     "simt": ("ssd_simt.cu", "ssd_internal.h"),
     "step": ("ssd_step.cu", "ssd_internal.h"),
@@ -754,8 +754,9 @@ def main():
                  else "fallback", "algorithmic_bytes_per_launch": byts,
                  "causal_flops_per_launch": flops, "tensor_tflops_achieved": achieved_tf,
                  "roofline_us": 1e6 * max(t_hbm, t_tc), "frac_of_roofline": 1e3 * max(t_hbm, t_tc) / ms,
-                 "kernel": traffic_kernel or {"tc": "ssd_tc_fused", "tc128": "ssd_tc_wide"}.get(
-                     path_name, "simt (4-5 kernels)")})
+                 "kernel": traffic_kernel or {"tc": "ssd_tc_fused<1>" if w.dstate <= 128
+                                              else "ssd_tc_fused2<2>",
+                                              "tc128": "ssd_tc_wide"}.get(path_name, "simt (4-5 kernels)")})
 
     # end to end through the host-buffer entry point (pinned host memory)
     host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in inp.items()}
