@@ -193,16 +193,21 @@ def oracle_sample_throughput(w, inp, budget_s):
                               heads=list(range(k)))
         return time.perf_counter() - t0
 
+    # the oracle runs its (sequence, head) items in parallel over its threads: size the
+    # head sample so that every thread is busy for about the budget
+    threads = oracle.oracle_threads()
+    seqs = int(inp["x"].shape[0]) if inp["cu_seqlens"] is None else int(inp["cu_seqlens"].numel() - 1)
     k = 1
     t = run(k)
     if t < 0.5 * budget_s and k < w.nheads:
-        k = int(min(w.nheads, max(1, round(k * budget_s / max(t, 1e-6)))))
+        waves = max(1, int(budget_s / max(t, 1e-6)))
+        k = int(min(w.nheads, max(1, (waves * threads) // max(seqs, 1))))
         t = run(k)
     reps = 1
     if t < 0.25 * budget_s:  # the whole workload is quick: repeat it
         reps = int(min(50, max(1, 0.5 * budget_s / max(t, 1e-6))))
         t = sum(run(k) for _ in range(reps)) / reps
-    return (w.tokens * k / w.nheads) / t / 1e6, k, t
+    return (w.tokens * k / w.nheads) / t / 1e6, k, t, min(threads, seqs * k)
 
 
 # ----------------------------------------------------------------------------- main
@@ -648,7 +653,7 @@ def main():
         import oracle
         inp = I.make_inputs(w, device="cpu")
         budget = max(0.05, min(10.0, 150.0 / (args.steps + args.warmup)))
-        _v, kh, _t = oracle_sample_throughput(w, inp, budget)
+        _v, kh, _t, ref_cores = oracle_sample_throughput(w, inp, budget)
         import oracle as _o
         cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].numpy()
 
@@ -672,7 +677,7 @@ def main():
             "ms_per_step": 1e3 * wall / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name},
-            "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": oracle.oracle_threads(),
+            "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": ref_cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
@@ -786,8 +791,8 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        v, kh, t = oracle_sample_throughput(w, inp, 12.0)
-        cpu = {"value": v, "unit": "Mtokens/s", "cores": oracle.oracle_threads(), "kind": "oracle",
+        v, kh, t, used = oracle_sample_throughput(w, inp, 12.0)
+        cpu = {"value": v, "unit": "Mtokens/s", "cores": used, "kind": "oracle",
                "sample": f"float64 oracle, heads 0..{kh - 1} of {w.nheads} over all {w.tokens} "
                          f"tokens in {t:.2f} s; whole-token throughput = tokens * {kh} / "
                          f"{w.nheads} / time"}
