@@ -314,8 +314,9 @@ def run_bwd(args, w, rank, world, local, pg, hbm_peak, tc_peak, peak_kind):
     Algorithmic flops per token and head, for chunks of Q tokens: 2 Q (2 P + 3 N)
     (the in-chunk products W, V, dC, dB, gB) + 8 N P (the state-sized products of
     dC, dB, gB and the per-chunk cotangent sum) + 2 N P (the forward's chunk states,
-    recomputed).  bf16 inputs with P = 64 and N = 64 or 128 take the tensor-core path
-    (Q = 128): its roofline is the measured bf16 tensor rate.  Every other shape runs
+    recomputed).  bf16 inputs with P a multiple of 64 (up to 256) and N = 64 or 128
+    take the tensor-core path (Q = 128, one block per 64-column slice of P): its
+    roofline is the measured bf16 tensor rate.  Every other shape runs
     on the CUDA cores (Q = 64) against the fp32 FMA rate, 148 SMs x 128 lanes x 2 x
     1965 MHz = 74.4 TFLOP/s.  L2 is flushed before every timed step.
     """
@@ -365,7 +366,7 @@ def run_bwd(args, w, rank, world, local, pg, hbm_peak, tc_peak, peak_kind):
     ms = statistics.median(a.elapsed_time(b) for a, b in zip(starts, ends))
     ms = max_over_ranks(pg, ms)
     T = bsz * L
-    on_tc = w.dtype == "bf16" and P == 64 and N in (64, 128)
+    on_tc = w.dtype == "bf16" and P % 64 == 0 and P <= 256 and N in (64, 128)
     Q = 128 if on_tc else 64
     flops = float(T) * H * (2 * Q * (2 * P + 3 * N) + 10 * N * P)
     if on_tc:
@@ -406,6 +407,8 @@ def run_bwd(args, w, rank, world, local, pg, hbm_peak, tc_peak, peak_kind):
                          "frac": achieved / peak, "traffic": None, "peak_source": peak_source,
                          "algorithmic_flops_per_launch": flops, "chunk": Q,
                          "kernel": ("kb_chunk_tc + kb_states_tc x2 + kb_state_pass + k_cumsum + k_state_pass"
+                                    if on_tc and N == 128 else
+                                    "kb_chunk_tc + kb_chunk_dstate + kb_state_pass + the forward's state kernels"
                                     if on_tc else
                                     "kb_chunk + kb_chunk_dstate + kb_state_pass + the forward's state kernels")},
             "cpu_baseline": cpu, "e2e": None, "gpu_launches": 11 * args.steps, "clocks": clocks,

@@ -231,12 +231,14 @@ SSD_API int ssd_forward_host(ssd_handle_t h, const void* x, const void* dt, cons
  *   (summed over the heads of each group); dA [H]; dD [H] and ddt_bias [H]
  *   (either may be NULL: not computed); dinitial_states [docs, H, N, P] or NULL.
  * The chunk size is the backward's own, whatever the forward used (the chunking
- * changes only rounding).  bf16 inputs and outputs with headdim 64, dstate 64 or
- * 128 and 16-byte aligned x, B, C, dy, dx, dB and dC run on the tensor cores with
- * 128-token chunks: bf16 operands, the in-chunk weighted matrices and the
- * cotangent as hi + lo bf16 pairs, fp32 accumulation.  Everything else runs on the
- * CUDA cores in fp32 with 64-token chunks.  dB, dC, dA, dD and ddt_bias are sums of
- * fp32 atomic additions, so their last bits can differ from run to run.  Workspace grows in the handle as for ssd_forward.  Errors as for
+ * changes only rounding).  bf16 inputs and outputs with headdim a multiple of 64
+ * (up to 256), dstate 64 or 128 and 16-byte aligned x, B, C, dy, dx, dB and dC run
+ * on the tensor cores with 128-token chunks, one slice of 64 head-dimension columns
+ * per block: bf16 operands, the in-chunk weighted matrices and the cotangent as
+ * hi + lo bf16 pairs, fp32 accumulation.  Everything else runs on the CUDA cores in
+ * fp32 with 64-token chunks.  dB, dC, dA, dD and ddt_bias (and ddt, when the head
+ * dimension has more than one slice) are sums of fp32 atomic additions, so their
+ * last bits can differ from run to run.  Workspace grows in the handle as for ssd_forward.  Errors as for
  * ssd_forward; inputs need only element alignment.
  */
 SSD_API int ssd_backward(ssd_handle_t h, const void* x, const void* dt, const float* A,

@@ -27,7 +27,7 @@
 //   kb_chunk         every per-token gradient of one (chunk, head) from 64 x 64 tiles
 //                    in shared memory; dB and dC add over the heads of a group
 //                    (fp32 atomics), dA, dD and ddt_bias over chunks.
-// For bf16 inputs with P = 64 and N = 64 or 128 (bwd_tc_eligible) the chunks are 128
+// For bf16 inputs with P a multiple of 64 (up to 256) and N = 64 or 128 (bwd_tc_eligible) the chunks are 128
 // tokens long and ssd_bwd_tc.cu takes over the products: kb_chunk_tc in place of
 // kb_chunk and, for N = 128, kb_states_tc in place of the two chunk-state products.
 #include <cuda_runtime.h>
@@ -476,6 +476,8 @@ cudaError_t bwd_run(const Geom& g, const Args& a_in, const GradArgs& ga, void* b
   zero(ga.dA, g.H);
   zero(ga.dD, g.H);
   zero(ga.ddt_bias, g.H);
+  // the tensor-core chunk kernel adds the parts of each 64-column slice of P into ddt
+  if (tc && g.P > 64) zero(ga.ddt, g.tokens * g.H);
   // the chunk-state products on the tensor cores when the chunk kernel is there and N = 128
   const bool tc_states = tc && g.N == 128;
   cudaError_t e;

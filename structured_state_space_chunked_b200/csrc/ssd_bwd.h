@@ -32,7 +32,7 @@ struct GradArgs {
   float* dinit;          // [ndocs, H, N, P] or null
 };
 
-// Chunk length of the tensor-core backward (bf16 inputs and outputs, P = 64, N = 64 or
+// Chunk length of the tensor-core backward (bf16 inputs and outputs, P a multiple of 64 up to 256, N = 64 or
 // 128, 16-byte aligned x, dy, B and C); ssd_backward takes it when bwd_tc_eligible.
 constexpr int kBwdTcQ = 128;
 bool bwd_tc_eligible(const Geom& g, const Args& a, const GradArgs& ga);

@@ -2,9 +2,12 @@
 //
 // The same chunk-level derivative as ssd_bwd.cu's kb_chunk ("Transformers are SSMs",
 // paperlayer.ai summary: the block decomposition of §6, differentiated), for bf16
-// inputs with P = 64 and N = 64 or 128, on 128-token chunks.  One CTA of 256 threads
-// per (chunk, head); threads r and r + 128 own row r of every 128-row accumulator, each
-// half of its columns.  Every matrix
+// inputs with P a multiple of 64 and N = 64 or 128, on 128-token chunks.  One CTA of 256
+// threads per (chunk, head, 64-column slice of P); threads r and r + 128 own row r of
+// every 128-row accumulator, each half of its columns.  Every gradient is linear in the
+// slices of the head dimension (x, dy and the state's columns enter each term once), so a
+// slice's CTA computes its part of every sum over p (S1, dY Hc^T, X dE^T, <C, dC>,
+// <x, gB>, <dE, S_last>) and the parts meet in the global accumulators.  Every matrix
 // is staged once in shared memory as bf16 128-byte-swizzled panels and read by the
 // MMAs either K-major or MN-major:
 //
@@ -97,7 +100,8 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   // 256 threads: thread (r, half) owns row r of the accumulators and half of the columns
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, r = tid & (kQ - 1), half = tid >> 7;
   const int64_t k = blockIdx.x;
-  const int h = blockIdx.y;
+  // blockIdx.y: (head, 64-column slice of its head dimension)
+  const int nps = g.P / 64, h = (int)blockIdx.y / nps, pofs = ((int)blockIdx.y % nps) * 64;
   ChunkInfo ci;
   if (!chunk_info(g, kp.a.cu, kp.ws, k, &ci)) return;
   const int N = g.N, P = g.P, H = g.H, G = g.G, grp = h / (H / G), len = ci.len;
@@ -144,8 +148,8 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int i = i0 + u * 256 + tid, n = i >> 3, c = i & 7;
-      const float4* ph = reinterpret_cast<const float4*>(Hc + (int64_t)n * P + 8 * c);
-      const float4* pe = reinterpret_cast<const float4*>(dE + (int64_t)n * P + 8 * c);
+      const float4* ph = reinterpret_cast<const float4*>(Hc + (int64_t)n * P + pofs + 8 * c);
+      const float4* pe = reinterpret_cast<const float4*>(dE + (int64_t)n * P + pofs + 8 * c);
       hv[u][0] = __ldg(ph);
       hv[u][1] = __ldg(ph + 1);
       ev[u][0] = __ldg(pe);
@@ -179,8 +183,8 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   // until phase D)
   if (tid == 0) {
     mbar_expect_tx(bar_load, (uint32_t)(2 + 2 * np) * kPanel);
-    tma_2d(s_x, &tm_x, bar_load, h * P, (int)t0);
-    tma_2d(s_dy, &tm_dy, bar_load, h * P, (int)t0);
+    tma_2d(s_x, &tm_x, bar_load, h * P + pofs, (int)t0);
+    tma_2d(s_dy, &tm_dy, bar_load, h * P + pofs, (int)t0);
     for (int q = 0; q < np; ++q) {
       tma_3d(s_b + q * kPanel, &tm_b, bar_load, 64 * q, grp, (int)t0);
       tma_3d(s_c + q * kPanel, &tm_c, bar_load, 64 * q, grp, (int)t0);
@@ -387,7 +391,7 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
       tc_ld32(trow + 64 + c0, b);
       tc_wait_ld();
       if (r < len) {
-        float4* dst = reinterpret_cast<float4*>(kp.ga.dx + ((t0 + r) * H + h) * (int64_t)P + c0);
+        float4* dst = reinterpret_cast<float4*>(kp.ga.dx + ((t0 + r) * H + h) * (int64_t)P + pofs + c0);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float xv[8], yv[8], o[8];
@@ -418,16 +422,17 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
     const int64_t cnt = doc_chunks(g, kp.ws, ci.doc, &first);
     const float* Hend = (k == first + cnt - 1) ? kp.bw.final + ((int64_t)ci.doc * H + h) * NP
                                                : kp.ws.states + ((k + 1) * H + h) * NP;
-    // 16-byte loads, eight in flight per thread
+    // over this CTA's 64 columns: 16-byte loads, eight in flight per thread (16 per
+    // state row; N * 16 is a multiple of 1024)
     float sp = 0.f;
-    const float4* d4 = reinterpret_cast<const float4*>(dE);
-    const float4* h4 = reinterpret_cast<const float4*>(Hend);
-    for (int64_t e0 = tid; e0 < NP / 4; e0 += 4 * 256) {
+    for (int e0 = tid; e0 < N * 16; e0 += 4 * 256) {
       float4 dv[4], hv[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        dv[u] = __ldg(d4 + e0 + u * 256);
-        hv[u] = __ldg(h4 + e0 + u * 256);
+        const int e = e0 + u * 256;
+        const int64_t off = (int64_t)(e >> 4) * P + pofs + 4 * (e & 15);
+        dv[u] = __ldg(reinterpret_cast<const float4*>(dE + off));
+        hv[u] = __ldg(reinterpret_cast<const float4*>(Hend + off));
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u)
@@ -467,7 +472,11 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
       const float ddelta = fmaf(kp.a.A[h], vdcs[tid], vxg[tid]);
       const float z = load_f(kp.a.dt, t * H + h, g.in_bf16) + (kp.a.dt_bias ? kp.a.dt_bias[h] : 0.f);
       const float gdt = ddelta / (1.f + expf(-z));
-      kp.ga.ddt[t * H + h] = gdt;
+      // every term is linear in the head-dimension slices: their parts add up
+      if (nps == 1)
+        kp.ga.ddt[t * H + h] = gdt;
+      else
+        atomicAdd(kp.ga.ddt + t * H + h, gdt);
       pA = vdl[tid] * vdcs[tid];
       pb = gdt;
     }
@@ -492,7 +501,8 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   }
 }
 
-// Chunk-state products on the tensor cores (N = 128, P = 64): D[n][p] = sum_t M[t][n] w_t V[t][p]
+// Chunk-state products on the tensor cores (N = 128, P a multiple of 64, one CTA per
+// 64-column slice): D[n][p] = sum_t M[t][n] w_t V[t][p]
 // with (M, V, w) = (B, x, exp(cs_last - cs_t) delta_t) for the forward's chunk states and
 // (C, dy, exp(cs_t)) for the cotangent sums.  The weighted rows w_t V[t] enter as hi + lo
 // bf16 pairs (about 16 bits), M as stored (bf16).  One CTA of 128 threads per (chunk,
@@ -506,7 +516,7 @@ __global__ void __launch_bounds__(128) kb_states_tc(const __grid_constant__ CUte
   const Geom& g = kp.g;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t k = blockIdx.x;
-  const int h = blockIdx.y;
+  const int nps = g.P / 64, h = (int)blockIdx.y / nps, pofs = ((int)blockIdx.y % nps) * 64;
   ChunkInfo ci;
   if (!chunk_info(g, kp.a.cu, kp.ws, k, &ci)) return;
   const int P = g.P, H = g.H, G = g.G, grp = h / (H / G), len = ci.len;
@@ -533,7 +543,7 @@ __global__ void __launch_bounds__(128) kb_states_tc(const __grid_constant__ CUte
     mbar_expect_tx(bar_load, 3 * kPanel);
     tma_3d(s_m, &tm_m, bar_load, 0, grp, (int)t0);
     tma_3d(s_m + kPanel, &tm_m, bar_load, 64, grp, (int)t0);
-    tma_2d(s_v, &tm_v, bar_load, h * P, (int)t0);
+    tma_2d(s_v, &tm_v, bar_load, h * P + pofs, (int)t0);
   }
   const int64_t cso = ((int64_t)h * g.nchunks_max + k) * g.Q;
   float w = 0.f;
@@ -568,7 +578,7 @@ __global__ void __launch_bounds__(128) kb_states_tc(const __grid_constant__ CUte
   if (ok) ok = wait_bar(bar_mma, 0, kp.status);
   tc_fence_after();
   if (ok) {
-    float* out = (mode == 0 ? kp.ws.states : kp.bw.dstates) + (k * H + h) * NP + (int64_t)tid * P;
+    float* out = (mode == 0 ? kp.ws.states : kp.bw.dstates) + (k * H + h) * NP + (int64_t)tid * P + pofs;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     for (int c0 = 0; c0 < 64; c0 += 32) {
       float a[32];
@@ -596,7 +606,7 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 }  // namespace
 
 bool bwd_tc_eligible(const Geom& g, const Args& a, const GradArgs& ga) {
-  return g.in_bf16 && g.out_bf16 && g.P == 64 && (g.N == 64 || g.N == 128) && aligned16(a.x) &&
+  return g.in_bf16 && g.out_bf16 && g.P % 64 == 0 && g.P <= 256 && (g.N == 64 || g.N == 128) && aligned16(a.x) &&
          aligned16(a.B) && aligned16(a.C) && aligned16(ga.dy) && aligned16(ga.dx) &&
          aligned16(ga.dB) && aligned16(ga.dC) && g.tokens <= 0x7fffffffLL;
 }
@@ -625,7 +635,8 @@ cudaError_t bwd_chunk_tc(const Geom& g, const Args& a, const GradArgs& ga, const
   const size_t smem = kb_chunk_tc_smem(g.N);
   cudaError_t e = cudaFuncSetAttribute(kb_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kb_chunk_tc<<<dim3((unsigned)g.nchunks_max, g.H), 256, smem, stream>>>(tm_x, tm_dy, tm_b, tm_c, kp);
+  kb_chunk_tc<<<dim3((unsigned)g.nchunks_max, g.H * (g.P / 64)), 256, smem, stream>>>(tm_x, tm_dy, tm_b, tm_c,
+                                                                                     kp);
   return cudaGetLastError();
 }
 
@@ -635,7 +646,7 @@ namespace ssd {
 
 cudaError_t bwd_states_tc(const Geom& g, const Args& a, const GradArgs& ga, const SimtWorkspace& ws,
                           const BwdWs& bw, int mode, int* status, cudaStream_t stream) {
-  if (g.Q != kQ || g.N != 128 || g.P != 64) return cudaErrorInvalidValue;
+  if (g.Q != kQ || g.N != 128 || g.P % 64 != 0) return cudaErrorInvalidValue;
   CUtensorMap tm_m, tm_v;
   const cuuint64_t T = (cuuint64_t)g.tokens;
   {
@@ -655,7 +666,7 @@ cudaError_t bwd_states_tc(const Geom& g, const Args& a, const GradArgs& ga, cons
   const size_t smem = 1024 + 5 * (size_t)kPanel;
   cudaError_t e = cudaFuncSetAttribute(kb_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kb_states_tc<<<dim3((unsigned)g.nchunks_max, g.H), 128, smem, stream>>>(tm_m, tm_v, kp, mode);
+  kb_states_tc<<<dim3((unsigned)g.nchunks_max, g.H * (g.P / 64)), 128, smem, stream>>>(tm_m, tm_v, kp, mode);
   return cudaGetLastError();
 }
 

@@ -512,9 +512,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : tst(HB_READY0, nds & 1))) {
           tc_fence_after();
           SSD_CHECK(dbg[DBG_BFILL + nds % C::BS] == (int)(nds / C::BS + 1), kp.status);
+          // (the count is raised before the issue: the product's completion can be
+          // observed before this warp would reach a store after it)
+          if (SSD_DEBUG_ON && lane == 0) dbg[DBG_NDS] = (int)nds + 1;
           if (nds & 1) issue_ds(I1{}); else issue_ds(I0{});
           ++nds;
-          if (SSD_DEBUG_ON && lane == 0) dbg[DBG_NDS] = (int)nds;
           did = true;
         } else if (nyo < ntiles && tst(HB_READY0 + nyo % C::HBS, (nyo / C::HBS) & 1) &&
                    tst(BCFULL0 + nyo % C::BS, (nyo / C::BS) & 1) &&
@@ -528,9 +530,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           // the B/C slot holds this tile's fill, not an earlier one
           SSD_CHECK(dbg[DBG_BFILL + ncb % C::BS] == (int)(ncb / C::BS + 1), kp.status);
+          if (SSD_DEBUG_ON && lane == 0) dbg[DBG_NCB] = (int)ncb + 1;
           if (ncb & 1) issue_cb(I1{}); else issue_cb(I0{});
           ++ncb;
-          if (SSD_DEBUG_ON && lane == 0) dbg[DBG_NCB] = (int)ncb;
           did = true;
         } else if (nyd < ncb && tst(M_READY0 + (nyd & 1), (nyd >> 1) & 1) &&
                    tst(XFULL0 + nyd % C::XS, (nyd / C::XS) & 1)) {

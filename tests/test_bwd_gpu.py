@@ -10,8 +10,10 @@ for the per-token gradients and the initial-state gradient, as for the forward's
 outputs; 1e-3 for dA, dD and dt_bias, each a sum over every token of the head whose
 terms cancel (the sum can be much smaller than its largest terms, and fp32 atomics add
 them in any order).  bf16 inputs: 2e-2 for every gradient, as for the forward's bf16
-path -- with P = 64 and N = 64 or 128 the in-chunk products run on the tensor cores
-with bf16 operands (the weighted matrices W' and V and the states rounded to bf16).
+path -- with P a multiple of 64 and N = 64 or 128 the in-chunk products run on the
+tensor cores with bf16 operands (the weighted matrices W' and V and the states rounded
+to bf16), one block per 64-column slice of P whose parts of every sum over p add up in
+the gradients.
 """
 
 import numpy as np
@@ -69,13 +71,17 @@ SMALL = [
     ("bf16", 2, 700, 4, 64, 128, 2, "normal0.1", 0),
     ("bf16", 1, 300, 2, 32, 64, 1, "normal0.1", 0),
     ("bf16", 1, 0, 4, 64, 128, 1, "normal0.1", 3000),
+    ("bf16", 2, 300, 4, 128, 128, 2, "normal0.1", 0),
+    ("bf16", 1, 0, 4, 128, 64, 2, "normal0.1", 1500),
+    ("bf16", 1, 270, 2, 192, 128, 1, "normal0.1", 0),
 ]
 
 
 @pytest.mark.parametrize("case", SMALL, ids=["fp32-G2", "bf16", "tiny-P16N16", "ragged-P80N72",
                                               "one-chunk-N256", "bf16-packed", "one-token",
                                               "bf16-G2-L700", "bf16-P32-cudacores",
-                                              "bf16-packed-N128"])
+                                              "bf16-packed-N128", "bf16-P128-tc", "bf16-P128-N64-packed",
+                                              "bf16-P192-tc"])
 def test_backward_matches_oracle(case):
     dtype, b, L, H, P, N, G, init, vt = case
     w = I.random_small(300 + P + N + L, dtype, b, L, H, P, N, G, 64, init, vt)
@@ -124,7 +130,8 @@ def test_only_final_state_cotangent_gives_the_pure_decay():
 
 
 @pytest.mark.parametrize("name,heads", [("mamba2_130m_layer_b4_L2048", [0, 13, 23]),
-                                        ("mamba2_2p7b_layer_b8_L4096", [5, 79])])
+                                        ("mamba2_2p7b_layer_b8_L4096", [5, 79]),
+                                        ("long_L16384_H64_P128_N128_G8", [0, 37, 63])])
 def test_backward_full_size_sampled_heads(name, heads):
     w = I.workload(name)
     inp = make(w)
