@@ -121,6 +121,14 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
     mbar_init(bar_load, 1);
     mbar_init(bar_mma, 1);
     fence_barrier_init();
+    // X, dY, B and C load while the threads convert the states below
+    mbar_expect_tx(bar_load, (uint32_t)(2 + 2 * np) * kPanel);
+    tma_2d(s_x, &tm_x, bar_load, h * P + pofs, (int)t0);
+    tma_2d(s_dy, &tm_dy, bar_load, h * P + pofs, (int)t0);
+    for (int q = 0; q < np; ++q) {
+      tma_3d(s_b + q * kPanel, &tm_b, bar_load, 64 * q, grp, (int)t0);
+      tma_3d(s_c + q * kPanel, &tm_c, bar_load, 64 * q, grp, (int)t0);
+    }
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&tslot)),
@@ -142,23 +150,37 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   // the entering state and the end-of-chunk cotangent as bf16 operands (rows n)
   const float* Hc = kp.ws.states + (k * H + h) * NP;
   const float* dE = kp.bw.dstates + (k * H + h) * NP;
+  // the state after the chunk (the next chunk's entering state, or the final state),
+  // for <dE, S_last>, summed here over this thread's elements while dE is in registers
+  int64_t first;
+  const int64_t cnt = doc_chunks(g, kp.ws, ci.doc, &first);
+  const float* Hend = (k == first + cnt - 1) ? kp.bw.final + ((int64_t)ci.doc * H + h) * NP
+                                             : kp.ws.states + ((k + 1) * H + h) * NP;
+  float sp = 0.f;
   // two rows of 8 columns per thread per round, all loads issued before the stores
   for (int i0 = 0; i0 < N * 8; i0 += 2 * 256) {
-    float4 hv[2][2], ev[2][2];
+    float4 hv[2][2], ev[2][2], sv[2][2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int i = i0 + u * 256 + tid, n = i >> 3, c = i & 7;
-      const float4* ph = reinterpret_cast<const float4*>(Hc + (int64_t)n * P + pofs + 8 * c);
-      const float4* pe = reinterpret_cast<const float4*>(dE + (int64_t)n * P + pofs + 8 * c);
+      const int64_t off = (int64_t)n * P + pofs + 8 * c;
+      const float4* ph = reinterpret_cast<const float4*>(Hc + off);
+      const float4* pe = reinterpret_cast<const float4*>(dE + off);
+      const float4* ps = reinterpret_cast<const float4*>(Hend + off);
       hv[u][0] = __ldg(ph);
       hv[u][1] = __ldg(ph + 1);
       ev[u][0] = __ldg(pe);
       ev[u][1] = __ldg(pe + 1);
+      sv[u][0] = __ldg(ps);
+      sv[u][1] = __ldg(ps + 1);
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int i = i0 + u * 256 + tid, n = i >> 3, c = i & 7;
       const float4 h0 = hv[u][0], h1 = hv[u][1], e0 = ev[u][0], e1 = ev[u][1];
+      const float4 s0 = sv[u][0], s1 = sv[u][1];
+      sp += e0.x * s0.x + e0.y * s0.y + e0.z * s0.z + e0.w * s0.w + e1.x * s1.x + e1.y * s1.y +
+            e1.z * s1.z + e1.w * s1.w;
       st_shared_v4(s_hc + swz((uint32_t)n, (uint32_t)c), pack_bf16(h0.x, h0.y), pack_bf16(h0.z, h0.w),
                    pack_bf16(h1.x, h1.y), pack_bf16(h1.z, h1.w));
       uint32_t eh[4], el[4];
@@ -179,16 +201,9 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   bool ok = true;
   uint32_t mma_phase = 0;
 
-  // phase A: loads, then S1 = dY X^T (cols 0..127) and S2 = C B^T (cols 256..383, kept
+  // phase A: once the loads landed, S1 = dY X^T (cols 0..127) and S2 = C B^T (cols 256..383, kept
   // until phase D)
   if (tid == 0) {
-    mbar_expect_tx(bar_load, (uint32_t)(2 + 2 * np) * kPanel);
-    tma_2d(s_x, &tm_x, bar_load, h * P + pofs, (int)t0);
-    tma_2d(s_dy, &tm_dy, bar_load, h * P + pofs, (int)t0);
-    for (int q = 0; q < np; ++q) {
-      tma_3d(s_b + q * kPanel, &tm_b, bar_load, 64 * q, grp, (int)t0);
-      tma_3d(s_c + q * kPanel, &tm_c, bar_load, 64 * q, grp, (int)t0);
-    }
     if (wait_bar(bar_load, 0, kp.status)) {
       tc_fence_after();
       const uint32_t id = idesc(128, 128, 0, 0);
@@ -418,26 +433,6 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
 
   // E5: <dE, S_last>, dcs and its reverse cumsum, ddt, the per-head sums
   if (ok) {
-    int64_t first;
-    const int64_t cnt = doc_chunks(g, kp.ws, ci.doc, &first);
-    const float* Hend = (k == first + cnt - 1) ? kp.bw.final + ((int64_t)ci.doc * H + h) * NP
-                                               : kp.ws.states + ((k + 1) * H + h) * NP;
-    // over this CTA's 64 columns: 16-byte loads, eight in flight per thread (16 per
-    // state row; N * 16 is a multiple of 1024)
-    float sp = 0.f;
-    for (int e0 = tid; e0 < N * 16; e0 += 4 * 256) {
-      float4 dv[4], hv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e0 + u * 256;
-        const int64_t off = (int64_t)(e >> 4) * P + pofs + 4 * (e & 15);
-        dv[u] = __ldg(reinterpret_cast<const float4*>(dE + off));
-        hv[u] = __ldg(reinterpret_cast<const float4*>(Hend + off));
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        sp += dv[u].x * hv[u].x + dv[u].y * hv[u].y + dv[u].z * hv[u].z + dv[u].w * hv[u].w;
-    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sp += __shfl_xor_sync(0xffffffffu, sp, o);
     if (lane == 0) red[warp] = sp;
