@@ -154,11 +154,12 @@ __global__ void __launch_bounds__(256)
 // to 256).  Work item = (b, h, column block of Pc <= 128 state columns, a run of
 // 128-token tiles); a persistent grid strides over the items.  Per item the CTA
 // writes its block of H_in once as a bf16 MN-major operand (state rows n are K).
-// Per tile: TMA brings the C tile and the y tile into shared memory, one thread
-// issues C H_in into TMEM (M = 128 tokens, N = Pc, K = dstate), two threads per token
-// row add exp(cs_t) times their halves of its accumulator row to its y row in shared
-// memory, and a TMA store writes the y tile back (rows past the slice are clipped by
-// the store).
+// Per tile: TMA brings the C tile into shared memory (the next one loads while this
+// tile's epilogue runs), one thread issues C H_in into TMEM (M = 128 tokens, N = Pc,
+// K = dstate), two threads per token row scale their halves of its accumulator row
+// by exp(cs_t) and stage them in y's type, and a TMA reduction adds the staged tile
+// into y (rows past the slice are clipped).  y is never read by the CTA: the addition
+// happens in L2, so no load of y sits in the tile's chain.
 constexpr int kCorrTile = 128;
 struct CorrParams {
   int64_t L;
@@ -186,6 +187,14 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t ph, int* statu
     }
   }
   return true;
+}
+
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, uint32_t src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
 }
 
 __global__ void __launch_bounds__(256)
@@ -227,14 +236,24 @@ __global__ void __launch_bounds__(256)
   const uint32_t id = idesc(128, p.Pc, 0, 1);
   const uint64_t dc = sdesc(sbase, 16, 1024), dh = sdesc(sbase + off_hb, hb_panel, 1024);
   const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-  uint32_t it = 0;  // tiles done by this CTA: the barriers' phase
+  // C tiles are loaded one ahead: the load of tile it (this CTA's count) completes
+  // phase it of `full`; nload counts the loads issued (thread 0)
+  uint32_t it = 0, nload = 0;
   bool ok = true;
+  auto load_c = [&](int g, int64_t row0) {
+    mbar_expect_tx(full, c_bytes);
+    for (int q = 0; q < npanel; ++q) tma_3d(sbase + q * kPanel, &tm_c, full, 64 * q, g, (int)row0);
+    ++nload;
+  };
   for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
     const int unit = item / p.items_per_unit;        // (b, h, column block)
     const int tile0 = (item % p.items_per_unit) * p.chunk;
     const int tile1 = min(p.ntiles, tile0 + p.chunk);
     const int pb = unit % nblk, bh = unit / nblk;
     const int b = bh / p.H, h = bh % p.H, g = h / (p.H / p.G);
+    // the item's first C tile loads while the state block converts (the previous
+    // item's products have completed: every tile waited on `done`)
+    if (threadIdx.x == 0) load_c(g, (int64_t)b * p.L + (int64_t)tile0 * kCorrTile);
     // this block of H_in as bf16: row n, 64-column panels, 128-byte swizzle
     const float* hsrc = p.h_in + (int64_t)bh * p.N * p.P + pb * p.Pc;
     for (int i = threadIdx.x; i < p.N * (p.Pc / 8); i += blockDim.x) {
@@ -250,12 +269,6 @@ __global__ void __launch_bounds__(256)
       const uint32_t ph = it & 1u;
       const int t0 = j * kCorrTile;
       if (threadIdx.x == 0) {
-        bulk_wait_read0();  // the previous tile's store has left the y buffer
-        mbar_expect_tx(full, c_bytes + y_bytes);
-        for (int q = 0; q < npanel; ++q)
-          tma_3d(sbase + q * kPanel, &tm_c, full, 64 * q, g, (int)(b * p.L + t0));
-        for (int q = 0; q < ypanels; ++q)
-          tma_3d(sbase + off_y + q * kPanel, &tm_y, full, h * p.P + pb * p.Pc + q * ycols, t0, b);
         if (wait_phase(full, ph, p.status)) {
           tc_fence_after();
           for (int kk = 0; kk < p.N / 16; ++kk)
@@ -265,10 +278,15 @@ __global__ void __launch_bounds__(256)
           ok = false;
         }
         tc_commit(done);  // arrives even when nothing was issued
+        bulk_wait_read0();  // the previous tile's reduction has read the staging tile
       }
-      ok = wait_phase(full, ph, p.status) && ok;
+      ok = __syncthreads_and(ok);
       ok = wait_phase(done, ph, p.status) && ok;
+      // the products have read C: the next tile's C tile loads during this epilogue
+      if (threadIdx.x == 0 && ok && j + 1 < tile1) load_c(g, (int64_t)b * p.L + t0 + kCorrTile);
       tc_fence_after();
+      // the correction exp(cs_t) (C_t H_in), in y's type, staged for a TMA reduction
+      // (addition) into y
       const int64_t t = (int64_t)t0 + r;
       const float e = (ok && t < p.L) ? expf(p.cs[((int64_t)b * p.L + t) * p.H + h]) : 0.f;
       for (int c0 = half * (p.Pc / 2); c0 < (half + 1) * (p.Pc / 2); c0 += 32) {
@@ -278,42 +296,37 @@ __global__ void __launch_bounds__(256)
         if (p.out_bf16) {
           const uint32_t row = sbase + off_y + (c0 >> 6) * kPanel;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t ad = row + swz((uint32_t)r, (uint32_t)(((c0 & 63) >> 3) + k));
-            uint4 v = ld_shared_v4(ad);
-            uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              const float lo = __uint_as_float(w[m] << 16), hi = __uint_as_float(w[m] & 0xffff0000u);
-              w[m] = pack_bf16(fmaf(e, acc[8 * k + 2 * m], lo), fmaf(e, acc[8 * k + 2 * m + 1], hi));
-            }
-            st_shared_v4(ad, w[0], w[1], w[2], w[3]);
-          }
+          for (int k = 0; k < 4; ++k)
+            st_shared_v4(row + swz((uint32_t)r, (uint32_t)(((c0 & 63) >> 3) + k)),
+                         pack_bf16(e * acc[8 * k], e * acc[8 * k + 1]), pack_bf16(e * acc[8 * k + 2], e * acc[8 * k + 3]),
+                         pack_bf16(e * acc[8 * k + 4], e * acc[8 * k + 5]),
+                         pack_bf16(e * acc[8 * k + 6], e * acc[8 * k + 7]));
         } else {
           const uint32_t row = sbase + off_y + (c0 >> 5) * kPanel;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t ad = row + swz((uint32_t)r, (uint32_t)k);
-            const uint4 v = ld_shared_v4(ad);
-            st_shared_v4(ad, __float_as_uint(fmaf(e, acc[4 * k], __uint_as_float(v.x))),
-                         __float_as_uint(fmaf(e, acc[4 * k + 1], __uint_as_float(v.y))),
-                         __float_as_uint(fmaf(e, acc[4 * k + 2], __uint_as_float(v.z))),
-                         __float_as_uint(fmaf(e, acc[4 * k + 3], __uint_as_float(v.w))));
-          }
+          for (int k = 0; k < 8; ++k)
+            st_shared_v4(row + swz((uint32_t)r, (uint32_t)k), __float_as_uint(e * acc[4 * k]),
+                         __float_as_uint(e * acc[4 * k + 1]), __float_as_uint(e * acc[4 * k + 2]),
+                         __float_as_uint(e * acc[4 * k + 3]));
         }
       }
-      fence_async_smem();  // the updated y tile is read by the TMA store
+      fence_async_smem();  // the staged tile is read by the TMA reduction
       tc_fence_before();
       ok = __syncthreads_and(ok);
       tc_fence_after();
       if (threadIdx.x == 0 && ok) {
         for (int q = 0; q < ypanels; ++q)
-          tma_store_3d(&tm_y, sbase + off_y + q * kPanel, h * p.P + pb * p.Pc + q * ycols, t0, b);
+          tma_reduce_add_3d(&tm_y, sbase + off_y + q * kPanel, h * p.P + pb * p.Pc + q * ycols, t0, b);
         bulk_commit();
       }
     }
   }
-  if (threadIdx.x == 0) bulk_wait0();
+  if (threadIdx.x == 0) {
+    bulk_wait0();
+    // the last C load has landed before shared memory goes (already true unless a
+    // wait ran out; bounded by time only)
+    if (nload > 0) wait_drain(full, (nload - 1) & 1u, 2000000000ull);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -438,8 +451,8 @@ extern "C" SSD_API int ssd_cp_correct(const ssd_desc_t* desc, const void* C, con
       const cuuint32_t box[3] = {(cuuint32_t)(128 / es), (cuuint32_t)ssd::kCorrTile, 1};
       if (!ssd::encode_sw128(&tm_y, ob, y, 3, dims, str, box)) return SSD_ERR_CUDA;
     }
-    // C tile, y tile, bf16 state block, alignment slack; never more CTAs on an SM
-    // than its 512 TMEM columns hold
+    // C tile, staged correction tile, bf16 state block, alignment slack; never more
+    // CTAs on an SM than its 512 TMEM columns hold
     size_t smem = 1024 + (size_t)(d.dstate / 64) * ssd::tc::kPanel + (size_t)Pc * es * ssd::kCorrTile +
                   (size_t)Pc * d.dstate * 2;
     const size_t per_sm = 228 * 1024, fit = (size_t)(512 / Pc);
