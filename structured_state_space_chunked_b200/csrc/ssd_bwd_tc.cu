@@ -157,26 +157,31 @@ __global__ void __launch_bounds__(256, 1) kb_chunk_tc(const __grid_constant__ CU
   const float* Hend = (k == first + cnt - 1) ? kp.bw.final + ((int64_t)ci.doc * H + h) * NP
                                              : kp.ws.states + ((k + 1) * H + h) * NP;
   float sp = 0.f;
-  // two rows of 8 columns per thread per round, all loads issued before the stores
-  for (int i0 = 0; i0 < N * 8; i0 += 2 * 256) {
-    float4 hv[2][2], ev[2][2], sv[2][2];
+  // every (row, 8 columns) piece of this thread (N * 8 / 256 of them: 4 for N = 128, 2 for
+  // N = 64) in one round, all loads issued before the stores
+  {
+    constexpr int kU = 4;
+    float4 hv[kU][2], ev[kU][2], sv[kU][2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i = i0 + u * 256 + tid, n = i >> 3, c = i & 7;
-      const int64_t off = (int64_t)n * P + pofs + 8 * c;
-      const float4* ph = reinterpret_cast<const float4*>(Hc + off);
-      const float4* pe = reinterpret_cast<const float4*>(dE + off);
-      const float4* ps = reinterpret_cast<const float4*>(Hend + off);
-      hv[u][0] = __ldg(ph);
-      hv[u][1] = __ldg(ph + 1);
-      ev[u][0] = __ldg(pe);
-      ev[u][1] = __ldg(pe + 1);
-      sv[u][0] = __ldg(ps);
-      sv[u][1] = __ldg(ps + 1);
+    for (int u = 0; u < kU; ++u) {
+      const int i = u * 256 + tid, n = i >> 3, c = i & 7;
+      if (i < N * 8) {
+        const int64_t off = (int64_t)n * P + pofs + 8 * c;
+        const float4* ph = reinterpret_cast<const float4*>(Hc + off);
+        const float4* pe = reinterpret_cast<const float4*>(dE + off);
+        const float4* ps = reinterpret_cast<const float4*>(Hend + off);
+        hv[u][0] = __ldg(ph);
+        hv[u][1] = __ldg(ph + 1);
+        ev[u][0] = __ldg(pe);
+        ev[u][1] = __ldg(pe + 1);
+        sv[u][0] = __ldg(ps);
+        sv[u][1] = __ldg(ps + 1);
+      }
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i = i0 + u * 256 + tid, n = i >> 3, c = i & 7;
+    for (int u = 0; u < kU; ++u) {
+      const int i = u * 256 + tid, n = i >> 3, c = i & 7;
+      if (i >= N * 8) continue;
       const float4 h0 = hv[u][0], h1 = hv[u][1], e0 = ev[u][0], e1 = ev[u][1];
       const float4 s0 = sv[u][0], s1 = sv[u][1];
       sp += e0.x * s0.x + e0.y * s0.y + e0.z * s0.z + e0.w * s0.w + e1.x * s1.x + e1.y * s1.y +
