@@ -98,3 +98,25 @@ def test_correction_equals_its_definition(P, N, G, L, out, tc):
     assert int(status.item()) == 0
     err = (yd.double().cpu() - ref).abs().max() / ref.abs().max()
     assert err <= (2e-2 if out == torch.bfloat16 else 1e-4)
+
+
+@pytest.mark.parametrize("out", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_correction_with_several_items_per_cta(out):
+    """Enough (batch, head, tile run) items that each persistent CTA of the tensor-core
+    correction takes several in a row (its C-tile prefetch and barrier phases carry
+    across items), against the definition in float64."""
+    g = torch.Generator().manual_seed(777)
+    b, L, H, P, N, G = 4, 2048, 48, 64, 128, 1
+    C = torch.randn(b, L, G, N, generator=g).to(torch.bfloat16)
+    cs = -torch.rand(b, L, H, generator=g).cumsum(1) * 0.002
+    h_in = torch.randn(b, H, N, P, generator=g)
+    y = torch.randn(b, L, H, P, generator=g).to(out)
+    ref = y.double() + cs.double().exp()[..., None] * torch.einsum(
+        "blhn,bhnp->blhp", C.double().expand(b, L, H, N), h_in.to(torch.bfloat16).double())
+    yd = y.cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ssd.cp_correct(C.cuda(), cs.cuda(), h_in.cuda(), yd, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    err = (yd.double().cpu() - ref).abs().max() / ref.abs().max()
+    assert err <= (2e-2 if out == torch.bfloat16 else 1e-4)
