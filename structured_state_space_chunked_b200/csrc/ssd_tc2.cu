@@ -30,9 +30,14 @@
 // Warps: 0-3 the state chain (S; also w o x, the B operand of dS), 4-7 and 8-11
 // two epilogue groups taking alternate tiles (cumulative decay, the decay mask
 // written over C B^T in TMEM as bf16, the outputs), 12 the MMA issuer and TMEM
-// owner, 13 the TMA producer.  The issuer and producer warps run their loops with all 32 lanes and
-// warp-uniform state; an elect.sync inside each instruction's asm block picks the
-// lane that issues it, so descriptors and coordinates stay in uniform registers.  Every mbarrier wait is bounded; a wait that runs out records
+// owner, 13 the TMA producer of B and C, 14 the TMA producer of x (a warp of its own,
+// so a wait for an x slot never holds up a B/C fill).  For N = 256 B and C sit in
+// separate 64 KB slots: C B^T of a tile is issued first, then dS (after which B's slot
+// frees, so the next tile's B loads while this tile's left factors run), then the left
+// factors (after which C's slot frees).  The issuer and producer warps run their loops
+// with all 32 lanes and warp-uniform state; a predicate inside each instruction's asm
+// block picks the lane that issues it, so descriptors and coordinates stay in uniform
+// registers.  Every mbarrier wait is bounded; a wait that runs out records
 // SSD_ERR_TIMEOUT in the status word, raises the CTA's abort flag and every role
 // unwinds; before TMEM is freed the issuer waits (bounded by time only) for its
 // products, and the producer for its loads.
@@ -52,7 +57,7 @@ using namespace tc;
 constexpr int kTile = 128;      // tokens per tile
 constexpr int kPT = 64;         // head-dim columns per unit
 constexpr int kThreads = 512;   // 16 warps
-constexpr int kWarpE0 = 4, kWarpE1 = 8, kWarpMma = 12, kWarpTma = 13;
+constexpr int kWarpE0 = 4, kWarpE1 = 8, kWarpMma = 12, kWarpTma = 13, kWarpX = 14;
 constexpr uint32_t kBarS = 3;   // named barrier of the state warpgroup (1, 2: epilogue groups)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -373,11 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t ntiles = count_tiles(kp);
 
-  if (warp == kWarpTma) {
-    // ================================ TMA producer ================================
+  if (warp == kWarpX) {
+    // ============================== TMA producer: x ==============================
     // The whole warp walks the stream (its values stay warp-uniform); one elected
     // lane issues each copy.
-    uint32_t nx = 0, nbc = 0;
+    uint32_t nx = 0;
     for (Cursor c = cursor_first(kp); c.valid; cursor_next(kp, c)) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const int t0 = (int)(c.U.start + (int64_t)c.jt * kTile);
@@ -393,6 +398,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_2d_w(sbase + C::OFF_X + s * C::X_BYTES, &tm_x, bar(XFULL0 + s), c.U.h * g.P + c.U.ps * kPT, t0);
         ++nx;
       }
+    }
+    for (uint32_t s = 0; s < (uint32_t)C::XS; ++s) {
+      if (nx <= s) continue;
+      const uint32_t last = (nx - 1 - s) / C::XS * C::XS + s;
+      wait_drain(bar(XFULL0 + s), (last / C::XS) & 1, 100000000ull);
+    }
+  } else if (warp == kWarpTma) {
+    // ============================= TMA producer: B, C =============================
+    // The whole warp walks the stream (its values stay warp-uniform); one elected
+    // lane issues each copy.
+    uint32_t nbc = 0;
+    for (Cursor c = cursor_first(kp); c.valid; cursor_next(kp, c)) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const int t0 = (int)(c.U.start + (int64_t)c.jt * kTile);
+      if constexpr (NT == 2) {
+        // B and C in separate slots: B frees once dS and C B^T read it, C once Yoff and
+        // C B^T did, so the next tile's B loads while this tile's Yoff runs
+        const uint32_t st = sbase + C::OFF_BC;
+        const int gi = c.U.h / (g.H / g.G);
+        if (nbc >= 1 && !__all_sync(0xffffffffu, waitb(BCEMPTY0, (nbc - 1) & 1))) break;
+        if (SSD_DEBUG_ON) {
+          if (lane == 0) dbg[DBG_BFILL] = (int)(nbc + 1);
+          __threadfence_block();
+        }
+        mbar_expect_tx_w(bar(BCFULL0), C::BC1_BYTES);
+#pragma unroll
+        for (int q = 0; q < C::NPANEL; ++q) tma_3d_w(st + q * kPanel, &tm_b, bar(BCFULL0), q * 64, gi, t0);
+        if (nbc >= 1 && !__all_sync(0xffffffffu, waitb(BCEMPTY1, (nbc - 1) & 1))) break;
+        if (SSD_DEBUG_ON) {
+          if (lane == 0) dbg[DBG_BFILL + 1] = (int)(nbc + 1);
+          __threadfence_block();
+        }
+        mbar_expect_tx_w(bar(BCFULL1), C::BC1_BYTES);
+#pragma unroll
+        for (int q = 0; q < C::NPANEL; ++q)
+          tma_3d_w(st + C::BC1_BYTES + q * kPanel, &tm_c, bar(BCFULL1), q * 64, gi, t0);
+        ++nbc;
+      } else
       {
         const uint32_t s = nbc % C::BS;
         if (nbc >= C::BS && !__all_sync(0xffffffffu, waitb(BCEMPTY0 + s, ((nbc - C::BS) / C::BS) & 1))) break;
@@ -412,23 +455,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++nbc;
       }
     }
-    // the last load into every slot has landed before the CTA frees anything
-    // (already true on the normal path; bounded by time on an aborted one)
-    for (uint32_t s = 0; s < (uint32_t)C::XS; ++s) {
-      if (nx <= s) continue;
-      const uint32_t last = (nx - 1 - s) / C::XS * C::XS + s;
-      wait_drain(bar(XFULL0 + s), (last / C::XS) & 1, 100000000ull);
-    }
-    for (uint32_t s = 0; s < (uint32_t)C::BS; ++s) {
-      if (nbc <= s) continue;
-      const uint32_t last = (nbc - 1 - s) / C::BS * C::BS + s;
-      wait_drain(bar(BCFULL0 + s), (last / C::BS) & 1, 100000000ull);
+    if constexpr (NT == 2) {
+      if (nbc > 0) {
+        wait_drain(bar(BCFULL0), (nbc - 1) & 1, 100000000ull);
+        wait_drain(bar(BCFULL1), (nbc - 1) & 1, 100000000ull);
+      }
+    } else {
+      for (uint32_t s = 0; s < (uint32_t)C::BS; ++s) {
+        if (nbc <= s) continue;
+        const uint32_t last = (nbc - 1 - s) / C::BS * C::BS + s;
+        wait_drain(bar(BCFULL0 + s), (last / C::BS) & 1, 100000000ull);
+      }
     }
   } else if (warp == kWarpMma) {
     // ================================ MMA issuer =================================
     // A non-blocking event loop over four in-order streams: dS (feeds the state
-    // chain), Yoff (left factors), C B^T, Ydiag.  A B/C slot is released once the
-    // three products that read it (dS, Yoff, C B^T) are issued.  The whole warp runs
+    // chain), Yoff (left factors), C B^T, Ydiag.  N <= 128: one product per pass, dS
+    // first, and a B/C slot is released once the three products that read it (dS,
+    // Yoff, C B^T) are issued.  N = 256: every ready product per pass in the order
+    // C B^T, dS, Yoff, Ydiag, each slot's commit straight after its last reader (a
+    // commit also waits for every MMA queued before it).  The whole warp runs
     // the loop with warp-uniform decisions and lane 0 issues each instruction.  Each
     // product is issued by a path specialised on the tile's parity, so every operand
     // is a loop-invariant base plus a compile-time offset.
@@ -498,11 +544,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       using I0 = std::integral_constant<uint32_t, 0>;
       using I1 = std::integral_constant<uint32_t, 1>;
-      uint32_t nds = 0, nyo = 0, ncb = 0, nyd = 0, nbc = 0, nxe = 0;
+      uint32_t nds = 0, nyo = 0, ncb = 0, nyd = 0, nbc = 0, nxe = 0, ncr = 0;
       uint64_t t_last = 0;
       uint32_t idle = 0;
       while (nyd < ntiles || nds < ntiles || nyo < ntiles) {
         bool did = false;
+        if constexpr (NT == 2) {
+          // C B^T first (it reads B and C), then dS (B), then Yoff (C): B's slot frees
+          // after dS, C's after Yoff
+          auto rel_b = [&]() {  // B read by C B^T and dS
+            while (nbc < nds && nbc < ncb) {
+              tc_commit_w(bar(BCEMPTY0));
+              ++nbc;
+            }
+          };
+          auto rel_x = [&]() {  // x read by Ydiag and (through w o x) dS
+            while (nxe < nyd && nxe < nds) {
+              tc_commit_w(bar(XEMPTY0 + nxe % C::XS));
+              ++nxe;
+            }
+          };
+          auto rel_c = [&]() {  // C read by C B^T and Yoff
+            while (ncr < nyo && ncr < ncb) {
+              tc_commit_w(bar(BCEMPTY1));
+              ++ncr;
+            }
+          };
+          if (ncb < ntiles && tst(BCFULL0, ncb & 1) && tst(BCFULL1, ncb & 1) &&
+              (ncb < 2 || tst(ZFREE0 + (ncb & 1), ((ncb - 2) >> 1) & 1))) {
+            tc_fence_after();
+            SSD_CHECK(dbg[DBG_BFILL] == (int)(ncb + 1) && dbg[DBG_BFILL + 1] == (int)(ncb + 1), kp.status);
+            if (SSD_DEBUG_ON && lane == 0) dbg[DBG_NCB] = (int)ncb + 1;
+            if (ncb & 1) issue_cb(I1{}); else issue_cb(I0{});
+            ++ncb;
+            did = true;
+            rel_b();
+            rel_c();
+          }
+          if (nds < ncb && tst(XW_READY0 + (nds & 1), (nds >> 1) & 1) && tst(HB_READY0, nds & 1)) {
+            tc_fence_after();
+            if (SSD_DEBUG_ON && lane == 0) dbg[DBG_NDS] = (int)nds + 1;
+            if (nds & 1) issue_ds(I1{}); else issue_ds(I0{});
+            ++nds;
+            did = true;
+            rel_b();  // straight after the issue: a later product's MMAs would hold the commit
+            rel_x();
+          }
+          if (nyo < ncb && tst(HB_READY0, nyo & 1) &&
+              (nyo < 2 || tst(ZFREE0 + (nyo & 1), ((nyo - 2) >> 1) & 1))) {
+            tc_fence_after();
+            if (nyo & 1) issue_yo(I1{}); else issue_yo(I0{});
+            ++nyo;
+            did = true;
+            rel_c();
+          }
+          if (nyd < ncb && tst(M_READY0 + (nyd & 1), (nyd >> 1) & 1) &&
+              tst(XFULL0 + nyd % C::XS, (nyd / C::XS) & 1)) {
+            tc_fence_after();
+            SSD_CHECK(dbg[DBG_XFILL + nyd % C::XS] == (int)(nyd / C::XS + 1), kp.status);
+            if (nyd & 1) issue_yd(I1{}); else issue_yd(I0{});
+            ++nyd;
+            did = true;
+            rel_x();
+          }
+
+        } else {
         // N <= 128: dS goes to a fresh buffer the state warps have read out;
         // N = 256: it accumulates onto the state the state warps decayed (HB_READY)
         if (nds < ntiles && tst(XW_READY0 + (nds & 1), (nds >> 1) & 1) &&
@@ -552,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit_w(bar(XEMPTY0 + nxe % C::XS));
           ++nxe;
         }
+        }  // NT == 1
         if (did) {
           idle = 0;
           t_last = 0;
