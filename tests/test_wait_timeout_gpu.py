@@ -25,7 +25,8 @@ SSD_ERR_TIMEOUT = -4
     # batch, seqlen, H, P, N, G, Q
     (2, 640, 4, 64, 128, 1, 256),
     (1, 300, 2, 128, 64, 2, 128),
-], ids=["b2-L640-N128", "b1-L300-P128-N64"])
+    (2, 700, 4, 128, 256, 2, 256),
+], ids=["b2-L640-N128", "b1-L300-P128-N64", "b2-L700-P128-N256"])
 def test_forced_wait_runs_out_then_the_handle_computes_again(case):
     b, L, H, P, N, G, Q = case
     w = I.random_small(70 + L, "bf16", b, L, H, P, N, G, Q, "normal0.1")
