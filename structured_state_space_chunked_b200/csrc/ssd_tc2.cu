@@ -1,5 +1,5 @@
 // ssd_tc2.cu -- fused SSD forward on the sm_100a tensor cores with the running
-// state held in registers (tcgen05 + TMEM + TMA).
+// state owned by a warpgroup of its own (tcgen05 + TMEM + TMA).
 //
 // A work unit is (document, head, 64-wide slice of the head dimension P).  A
 // persistent CTA walks its units' tokens in tiles of 128.  For tile j of a unit
@@ -11,17 +11,18 @@
 //   M[l,s]   = Z[l,s] exp(cs_l - cs_s) delta_s,  s <= l;  M[l,l] += D
 //   Ydiag    = M x_j                                (tensor cores, M from TMEM)
 //   dS_j     = B_j^T (w o x_j),  w_s = exp(cs_last - cs_s) delta_s
-//                                                   (right factors, tensor cores,
-//                                                    into a fresh TMEM buffer)
+//                                                   (right factors, tensor cores)
 //   S_{j+1}  = exp(cs_last) S_j + dS_j              (the scan across tiles)
 //   Yoff     = C_j bf16(S_j)                        (left factors, tensor cores)
 //   y        = exp(cs_l) Yoff + Ydiag
 //
-// The recurrence across tiles is the only serial dependence.  Here it runs on
-// CUDA cores in registers: warpgroup S holds S (64 columns of N rows, fp32) and per
-// tile adds dS_j and writes the bf16 copy the next tile's left-factor product
-// reads.  No tensor-core product waits on the previous tile's state update, so
-// products of several tiles are in flight at once.  A chunk of Q = 128 or 256
+// The recurrence across tiles is the only serial dependence, and warpgroup S owns
+// it.  N <= 128: S sits in its registers (64 columns of N rows, fp32); per tile it
+// adds dS_j, which the tensor cores write into a fresh TMEM buffer, and writes the
+// bf16 copy the next tile's left-factor product reads, so no product waits on the
+// previous tile's update.  N = 256 (two 128-row lane tiles, too many registers): S
+// stays in TMEM; per tile the warpgroup writes its bf16 copy, decays it in place, and
+// the tensor cores accumulate dS_j onto it.  A chunk of Q = 128 or 256
 // tokens is processed as Q/128 tiles: for Q = 256 the strictly lower 128 x 128
 // block of the chunk's quadratic form goes through the same rank-N factorisation
 // the decomposition uses between chunks (the mask restricted to a strictly lower
