@@ -522,7 +522,8 @@ __global__ void __launch_bounds__(128) kb_states_tc(const __grid_constant__ CUte
   const int P = g.P, H = g.H, G = g.G, grp = h / (H / G), len = ci.len;
   const int64_t NP = (int64_t)g.N * P, t0 = ci.start;
   const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t s_m = sbase, s_v = s_m + 2 * kPanel, s_hi = s_v + kPanel, s_lo = s_hi + kPanel;
+  // the hi halves overwrite V in place (each thread reads its own row before writing it)
+  const uint32_t s_m = sbase, s_v = s_m + 2 * kPanel, s_hi = s_v, s_lo = s_v + kPanel;
   const uint32_t bar_load = su32(&bars[0]), bar_mma = su32(&bars[1]);
   if (tid == 0) {
     mbar_init(bar_load, 1);
@@ -663,7 +664,7 @@ cudaError_t bwd_states_tc(const Geom& g, const Args& a, const GradArgs& ga, cons
     if (!tc::encode_bf16_sw128(&tm_v, mode == 0 ? a.x : ga.dy, 2, dims, str, box)) return cudaErrorInvalidValue;
   }
   TcParams kp{g, a, ga, ws, bw, status};
-  const size_t smem = 1024 + 5 * (size_t)kPanel;
+  const size_t smem = 1024 + 4 * (size_t)kPanel;  // three CTAs per SM
   cudaError_t e = cudaFuncSetAttribute(kb_states_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kb_states_tc<<<dim3((unsigned)g.nchunks_max, g.H * (g.P / 64)), 128, smem, stream>>>(tm_m, tm_v, kp, mode);
