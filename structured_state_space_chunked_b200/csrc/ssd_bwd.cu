@@ -43,10 +43,22 @@ constexpr int kTileF = 64 * kLD;   // floats per tile
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-__global__ void kb_zero(float* p, int64_t n) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    p[i] = 0.f;
+// up to six arrays zeroed by one launch: the grid strides over their concatenation
+struct ZeroList {
+  float* p[6];
+  int64_t n[6];
+  int count;
+};
+__global__ void kb_zero(ZeroList z) {
+  int64_t total = 0;
+  for (int k = 0; k < z.count; ++k) total += z.n[k];
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t j = i;
+    int k = 0;
+    while (j >= z.n[k]) j -= z.n[k++];
+    z.p[k][j] = 0.f;
+  }
 }
 
 // dS_c[n][p] = sum_l exp(cs_l) C[l][n] dy[l][p] over the tokens of chunk c
@@ -465,10 +477,13 @@ cudaError_t bwd_run(const Geom& g, const Args& a_in, const GradArgs& ga, void* b
   a.y = nullptr;
   a.final_states = bw.final;
 
+  ZeroList zl{};
+  int64_t ztotal = 0;
   auto zero = [&](float* q, int64_t n) {
     if (q && n > 0) {
-      const int64_t blocks = (n + 255) / 256;
-      kb_zero<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(q, n);
+      zl.p[zl.count] = q;
+      zl.n[zl.count++] = n;
+      ztotal += n;
     }
   };
   zero(ga.dB, g.tokens * g.G * g.N);
@@ -478,6 +493,10 @@ cudaError_t bwd_run(const Geom& g, const Args& a_in, const GradArgs& ga, void* b
   zero(ga.ddt_bias, g.H);
   // the tensor-core chunk kernel adds the parts of each 64-column slice of P into ddt
   if (tc && g.P > 64) zero(ga.ddt, g.tokens * g.H);
+  if (ztotal > 0) {
+    const int64_t blocks = (ztotal + 255) / 256;
+    kb_zero<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(zl);
+  }
   // the chunk-state products on the tensor cores when the chunk kernel is there and N = 128
   const bool tc_states = tc && g.N == 128;
   cudaError_t e;
