@@ -43,21 +43,26 @@ constexpr int kTileF = 64 * kLD;   // floats per tile
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// up to six arrays zeroed by one launch: the grid strides over their concatenation
+// up to six arrays zeroed by one launch: array k takes blocks first[k] .. first[k+1] - 1,
+// each block a run of kZeroRun consecutive elements
+constexpr int kZeroRun = 256 * 8;
 struct ZeroList {
   float* p[6];
   int64_t n[6];
+  int64_t first[7];
   int count;
 };
-__global__ void kb_zero(ZeroList z) {
-  int64_t total = 0;
-  for (int k = 0; k < z.count; ++k) total += z.n[k];
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    int64_t j = i;
+__global__ void __launch_bounds__(256) kb_zero(ZeroList z) {
+  for (int64_t blk = blockIdx.x; blk < z.first[z.count]; blk += gridDim.x) {
     int k = 0;
-    while (j >= z.n[k]) j -= z.n[k++];
-    z.p[k][j] = 0.f;
+    while (blk >= z.first[k + 1]) ++k;
+    const int64_t base = (blk - z.first[k]) * kZeroRun;
+    float* q = z.p[k];
+#pragma unroll
+    for (int u = 0; u < kZeroRun / 256; ++u) {
+      const int64_t i = base + u * 256 + threadIdx.x;
+      if (i < z.n[k]) q[i] = 0.f;
+    }
   }
 }
 
@@ -478,12 +483,12 @@ cudaError_t bwd_run(const Geom& g, const Args& a_in, const GradArgs& ga, void* b
   a.final_states = bw.final;
 
   ZeroList zl{};
-  int64_t ztotal = 0;
   auto zero = [&](float* q, int64_t n) {
     if (q && n > 0) {
       zl.p[zl.count] = q;
-      zl.n[zl.count++] = n;
-      ztotal += n;
+      zl.n[zl.count] = n;
+      zl.first[zl.count + 1] = zl.first[zl.count] + (n + kZeroRun - 1) / kZeroRun;
+      ++zl.count;
     }
   };
   zero(ga.dB, g.tokens * g.G * g.N);
@@ -493,9 +498,9 @@ cudaError_t bwd_run(const Geom& g, const Args& a_in, const GradArgs& ga, void* b
   zero(ga.ddt_bias, g.H);
   // the tensor-core chunk kernel adds the parts of each 64-column slice of P into ddt
   if (tc && g.P > 64) zero(ga.ddt, g.tokens * g.H);
-  if (ztotal > 0) {
-    const int64_t blocks = (ztotal + 255) / 256;
-    kb_zero<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(zl);
+  if (zl.count > 0) {
+    const int64_t blocks = zl.first[zl.count];
+    kb_zero<<<(unsigned)(blocks < 8192 ? blocks : 8192), 256, 0, stream>>>(zl);
   }
   // the chunk-state products on the tensor cores when the chunk kernel is there and N = 128
   const bool tc_states = tc && g.N == 128;
