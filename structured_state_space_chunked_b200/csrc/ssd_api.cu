@@ -358,8 +358,7 @@ int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* 
   void* dws = base + 2 * b_bc + b_den + b_fwd;
   const int bf = d.in_dtype == SSD_BF16;
   const int64_t rows = tokens * d.ngroups;
-  cudaError_t e = ssd::fmap_apply(feature_map, rows, (int)d.dstate, N2, bf, B, B2, stream);
-  if (e == cudaSuccess) e = ssd::fmap_apply(feature_map, rows, (int)d.dstate, N2, bf, C, C2, stream);
+  cudaError_t e = ssd::fmap_apply(feature_map, rows, (int)d.dstate, N2, bf, B, B2, C, C2, stream);
   // the numerator (D added after the division when normalising)
   ssd::Args a{x, dt, A, B2, C2, normalize ? nullptr : D, dt_bias, nullptr, cu_seqlens, y, final_states};
   if (e == cudaSuccess) {

@@ -7,9 +7,10 @@ namespace ssd {
 
 // dstate after feature map `kind` (SSD_FMAP_*) of an N-wide input; -1 if unknown
 int fmap_dim(int kind, int N);
-// dst[r, :] = phi(src[r, :]) for rows r < rows; src rows N wide, dst rows Nout wide
-cudaError_t fmap_apply(int kind, int64_t rows, int N, int Nout, int bf16, const void* src, void* dst,
-                       cudaStream_t stream);
+// dstB[r, :] = phi(srcB[r, :]) and dstC[r, :] = phi(srcC[r, :]) for rows r < rows; source
+// rows N wide, mapped rows Nout wide
+cudaError_t fmap_apply(int kind, int64_t rows, int N, int Nout, int bf16, const void* srcB, void* dstB,
+                       const void* srcC, void* dstC, cudaStream_t stream);
 // y[t, h, :] = y[t, h, :] / den[t, h] + D[h] x[t, h, :]
 cudaError_t normalize_apply(int64_t T, int H, int P, int out_bf16, int in_bf16, void* y,
                             const float* den, const void* x, const float* D, cudaStream_t stream);

@@ -36,10 +36,17 @@ CASES = [
     ("bf16", 2, 520, 4, 64, 128, 2, ssd.SSD_FMAP_RELU, True, 0, 256),
     ("bf16", 1, 700, 2, 64, 8, 1, ssd.SSD_FMAP_REBASED, True, 0, 256),
     ("bf16", 1, 0, 4, 64, 8, 1, ssd.SSD_FMAP_REBASED, True, 1500, 256),
+    # the denominator's block form with full head blocks (24 heads of one group, as in
+    # the 130M layer), a ragged head block (12 heads per group: 8 + 4) over packed
+    # documents, and the largest mapped dstate it takes (256, fp32)
+    ("bf16", 2, 700, 24, 64, 128, 1, ssd.SSD_FMAP_RELU, True, 0, 256),
+    ("bf16", 1, 0, 24, 64, 64, 2, ssd.SSD_FMAP_RELU, True, 1300, 256),
+    ("fp32", 1, 300, 3, 16, 16, 1, ssd.SSD_FMAP_REBASED, True, 0, 64),
 ]
 IDS = ["silu-simt", "relu-norm-simt", "based-norm-simt-fp32", "rebased-norm-simt",
        "based-norm-packed-simt", "none-norm-fp32", "relu-fp32",
-       "silu-tc", "relu-norm-tc", "rebased-norm-tc", "rebased-norm-packed-tc"]
+       "silu-tc", "relu-norm-tc", "rebased-norm-tc", "rebased-norm-packed-tc",
+       "relu-norm-tc-h24", "relu-norm-packed-tc-hpg12", "rebased-norm-fp32-n256"]
 
 
 @pytest.mark.parametrize("case", CASES, ids=IDS)
