@@ -498,8 +498,9 @@ def run_ext(args, w, rank, world, local, pg, hbm_peak, peak_kind):
                          "frac": achieved / hbm_peak, "traffic": None,
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json burst)" if peak_kind == "measured"
                          else "fallback", "algorithmic_bytes_per_launch": byts,
-                         "kernel": "fmap_kernel x2 + ssd_tc_fused + den_chunk_gram_kernel x2 + den_pass_kernel + normalize_kernel"},
-            "cpu_baseline": None, "e2e": None, "gpu_launches": 5 * args.steps, "clocks": clocks,
+                         "kernel": "fmap_ew_kernel (B and C) + ssd_tc_fused, beside it on a second stream "
+                                   "den_chunk_gram_kernel x2 + den_pass_kernel; then normalize_kernel"},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": 6 * args.steps, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if pg is not None:

@@ -25,6 +25,10 @@ struct ssd_handle_s {
   size_t ws_bytes;
   void* io;             // device buffers of ssd_forward_host
   size_t io_bytes;
+  // ssd_forward_ext's second stream: the denominator runs there beside the numerator
+  // (forked after the feature maps, joined before the normalisation); made on first use
+  cudaStream_t side;
+  cudaEvent_t ev_fork, ev_join;
 };
 
 namespace {
@@ -359,6 +363,12 @@ int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* 
   const int bf = d.in_dtype == SSD_BF16;
   const int64_t rows = tokens * d.ngroups;
   cudaError_t e = ssd::fmap_apply(feature_map, rows, (int)d.dstate, N2, bf, B, B2, C, C2, stream);
+  if (normalize && e == cudaSuccess && !h->side) {
+    e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
+  }
+  if (normalize && e == cudaSuccess) e = cudaEventRecord(h->ev_fork, stream);
   // the numerator (D added after the division when normalising)
   ssd::Args a{x, dt, A, B2, C2, normalize ? nullptr : D, dt_bias, nullptr, cu_seqlens, y, final_states};
   if (e == cudaSuccess) {
@@ -371,7 +381,14 @@ int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* 
     }
   }
   if (normalize && e == cudaSuccess) {
-    e = ssd::den_scan(gd, cu_seqlens, dws, h->status, dt, A, dt_bias, B2, C2, den, stream);
+    // the denominator on the side stream, its chain beside the numerator's kernel
+    e = cudaStreamWaitEvent(h->side, h->ev_fork, 0);
+    if (e == cudaSuccess) e = ssd::den_scan(gd, cu_seqlens, dws, h->status, dt, A, dt_bias, B2, C2, den, h->side);
+    // the join is recorded even after a failed launch, so the caller's stream never waits on
+    // an event of an earlier call
+    const cudaError_t ej = cudaEventRecord(h->ev_join, h->side);
+    if (e == cudaSuccess) e = ej;
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, h->ev_join, 0);
     if (e == cudaSuccess)
       e = ssd::normalize_apply(tokens, (int)d.nheads, (int)d.headdim, d.out_dtype == SSD_BF16, bf, y,
                                den, x, D, stream);
@@ -499,6 +516,9 @@ int ssd_destroy(ssd_handle_t h) {
   }
   if (h->io) cudaFree(h->io);
   if (h->status) cudaFree(h->status);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->side) cudaStreamDestroy(h->side);
   if (cur != h->device) cudaSetDevice(cur);
   delete h;
   return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;

@@ -68,6 +68,10 @@ def test_forward_ext_matches_oracle(case):
                            cu_seqlens=inp["cu_seqlens"])
     assert h.status() == 0
     torch.cuda.synchronize()
+    check_against_oracle(dtype, inp, y, fin, fmap, norm, N)
+
+
+def check_against_oracle(dtype, inp, y, fin, fmap, norm, N):
     cu = None if inp["cu_seqlens"] is None else inp["cu_seqlens"].cpu().numpy()
     cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
     yr, fr = oracle.oracle_forward_ext(cpu["x"], cpu["dt"], cpu["A"], cpu["B"], cpu["C"], cpu["D"],
@@ -95,6 +99,29 @@ def test_forward_ext_matches_oracle(case):
     assert fin.shape[2] == ssd.feature_map_dim(fmap, N)
     ef = rel_err(to_np(fin), fr)
     assert ef <= tol, f"final_states rel err {ef:.3e}"
+
+
+
+def test_forward_ext_repeated_calls_on_one_handle():
+    """Three normalised calls on one handle (the denominator runs on the handle's second
+    stream), each checked against the oracle, with different inputs and a packed one."""
+    L, H, P, N, G = 1400, 24, 64, 128, 1
+    outs = []
+    h = None
+    for seed, vt in ((31, 0), (32, 0), (33, L)):
+        w = I.random_small(seed, "bf16", 1, 0 if vt else L, H, P, N, G, 256, "zero", vt)
+        inp = make(w)
+        assert inp["x"].shape[:2] == (1, L)
+        if h is None:
+            h = ssd.SSD(1, L, H, P, N, G, torch.bfloat16, max_docs=L)
+        y, fin = h.forward_ext(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"],
+                               inp["dt_bias"], 256, feature_map=ssd.SSD_FMAP_RELU, normalize=True,
+                               cu_seqlens=inp["cu_seqlens"])
+        outs.append((inp, y.clone(), fin.clone()))
+    torch.cuda.synchronize()
+    assert h.status() == 0
+    for inp, y, fin in outs:
+        check_against_oracle("bf16", inp, y, fin, ssd.SSD_FMAP_RELU, True, N)
 
 
 def test_unknown_feature_map_is_refused():
