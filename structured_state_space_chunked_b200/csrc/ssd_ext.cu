@@ -247,14 +247,6 @@ __device__ __forceinline__ void store_f4(float* d, uint4 q, float) {
   *reinterpret_cast<float4*>(d) = make_float4(__uint_as_float(q.x), __uint_as_float(q.y),
                                               __uint_as_float(q.z), __uint_as_float(q.w));
 }
-__device__ __forceinline__ void store_f4(float* d, uint4 q, __nv_bfloat16) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
-  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-  const float2 c = __bfloat1622float2(h[2]), e = __bfloat1622float2(h[3]);
-  *reinterpret_cast<float4*>(d) = make_float4(a.x, a.y, b.x, b.y);
-  *reinterpret_cast<float4*>(d + 4) = make_float4(c.x, c.y, e.x, e.y);
-}
-
 // Rows t < len (columns n < N) of a chunk's B (and C when TWO) into dst[t][n] as fp32,
 // zeros elsewhere in [64][NR].  Loads are issued in batches before any of them is
 // stored; 16-byte loads when vec (N a whole number of them and 16-byte-aligned bases).
@@ -318,61 +310,29 @@ __device__ __forceinline__ void stage_chunk_rows(float* dB, float* dC, int NS, c
 // addresses of an ldmatrix fall in distinct quads
 __host__ __device__ inline int gram_stride_h(int N) { return ((N + 31) & ~31) + 8; }
 
-// Rows t < len (columns n < N) of a chunk's B and C into dB[t][n], dC[t][n] as bf16, zeros
-// elsewhere in [64][NR]; 16-byte copies when vec.
-__device__ __forceinline__ void stage_chunk_rows_h(__nv_bfloat16* dB, __nv_bfloat16* dC, int NSh,
-                                                   const __nv_bfloat16* B, const __nv_bfloat16* C,
-                                                   int64_t row0, int64_t rstride, int len, int N, int NR,
-                                                   int vec, int tid) {
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Rows t < len (columns n < N) of a chunk's matrix into d[t][n] as bf16, zeros elsewhere in
+// [64][NR].  vec: asynchronous 16-byte copies (zero-filled past the rows and columns), all
+// in flight at once, completed by the caller's cp_async_wait_all; else element copies.
+__device__ __forceinline__ void stage_rows_h(__nv_bfloat16* d, int NSh, const __nv_bfloat16* src, int64_t row0,
+                                             int64_t rstride, int len, int N, int NR, int vec, int tid) {
   if (vec) {
-    constexpr int R = 4;
     const int vpr = NR / 8, total = kDenQ * vpr;
-    for (int base = tid; base < total; base += kGramThreads * R) {
-      uint4 qb[R], qc[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int i = base + r * kGramThreads, t = i / vpr, c = (i % vpr) * 8;
-        qb[r] = make_uint4(0u, 0u, 0u, 0u);
-        qc[r] = qb[r];
-        if (i < total && t < len && c < N) {
-          const int64_t off = row0 + t * rstride + c;
-          qb[r] = *reinterpret_cast<const uint4*>(B + off);
-          qc[r] = *reinterpret_cast<const uint4*>(C + off);
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int i = base + r * kGramThreads, t = i / vpr, c = (i % vpr) * 8;
-        if (i < total) {
-          *reinterpret_cast<uint4*>(dB + t * NSh + c) = qb[r];
-          *reinterpret_cast<uint4*>(dC + t * NSh + c) = qc[r];
-        }
-      }
+    const uint32_t d0 = static_cast<uint32_t>(__cvta_generic_to_shared(d));
+    for (int i = tid; i < total; i += kGramThreads) {
+      const int t = i / vpr, c = (i % vpr) * 8;
+      const bool ok = t < len && c < N;
+      cp_async16(d0 + (uint32_t)((t * NSh + c) * 2), ok ? src + row0 + t * rstride + c : src, ok ? 16 : 0);
     }
   } else {
-    constexpr int R = 8;
-    const int total = kDenQ * NR;
     const __nv_bfloat16 zero = __float2bfloat16(0.f);
-    for (int base = tid; base < total; base += kGramThreads * R) {
-      __nv_bfloat16 vb[R], vc[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int i = base + r * kGramThreads, t = i / NR, n = i % NR;
-        vb[r] = zero;
-        vc[r] = zero;
-        if (i < total && t < len && n < N) {
-          vb[r] = B[row0 + t * rstride + n];
-          vc[r] = C[row0 + t * rstride + n];
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int i = base + r * kGramThreads, t = i / NR, n = i % NR;
-        if (i < total) {
-          dB[t * NSh + n] = vb[r];
-          dC[t * NSh + n] = vc[r];
-        }
-      }
+    for (int i = tid; i < kDenQ * NR; i += kGramThreads) {
+      const int t = i / NR, n = i % NR;
+      d[t * NSh + n] = (t < len && n < N) ? src[row0 + t * rstride + n] : zero;
     }
   }
 }
@@ -398,12 +358,22 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// bytes of the staged B rows (bf16 pass 3): G is written over them once they are read
+__host__ __device__ inline size_t den_gram_rows_h(int N) {
+  const size_t rows = (size_t)kDenQ * gram_stride_h(N) * 2, g = (size_t)kDenQ * (kDenQ + 1) * 4;
+  return rows > g ? rows : g;
+}
+
 size_t den_gram_smem(int N, bool out, bool bf16) {
   const size_t NS = (size_t)gram_stride(N);
   size_t f = 2 * (size_t)kDenHeads * kDenQ;  // delta, cs
-  if (!out) return (f + (size_t)kDenQ * NS + (size_t)kDenHeads * kDenQ + (size_t)kDenHeads * kGramThreads) * 4;
+  if (!out) {
+    const size_t rows = bf16 ? (size_t)kDenQ * gram_stride_h(N) * 2 : (size_t)kDenQ * NS * 4;
+    return rows + (f + (size_t)kDenHeads * kDenQ + (size_t)kDenHeads * kGramThreads) * 4;
+  }
   f += (size_t)kDenQ * (kDenQ + 1) + (size_t)kDenQ * kDenHeads;  // G, <C, z_in>
-  if (bf16) return (f + (size_t)kDenHeads * NS) * 4 + 2 * (size_t)kDenQ * gram_stride_h(N) * 2;
+  if (bf16) return (2 * (size_t)kDenHeads * kDenQ + (size_t)kDenHeads * NS) * 4 + den_gram_rows_h(N) +
+                   (size_t)kDenQ * gram_stride_h(N) * 2;
   return (f + (size_t)(2 * kDenQ + kDenHeads) * NS) * 4;
 }
 
@@ -416,10 +386,13 @@ __global__ void __launch_bounds__(kGramThreads)
   constexpr bool kH = sizeof(TIn) == 2;
   const int N = g.N, NR = (N + 31) & ~31, NS = gram_stride(N), tid = threadIdx.x, w = tid >> 5,
             lane = tid & 31;
-  const int hpg = g.H / g.G, hblocks = (hpg + kDenHeads - 1) / kDenHeads;
-  const int grp = (int)blockIdx.y / hblocks, hb0 = ((int)blockIdx.y % hblocks) * kDenHeads;
+  // the head blocks of one chunk are consecutive blocks, so they run together and share
+  // the chunk's B and C rows in L2
+  const int hpg = g.H / g.G, hblocks = (hpg + kDenHeads - 1) / kDenHeads, nhb = g.G * hblocks;
+  const int64_t lin = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+  const int64_t k = lin / nhb;
+  const int hb = (int)(lin % nhb), grp = hb / hblocks, hb0 = (hb % hblocks) * kDenHeads;
   const int nh = min(kDenHeads, hpg - hb0), h0 = grp * hpg + hb0;
-  const int64_t k = blockIdx.x;
   ChunkInfo ci;
   if (!chunk_info(g, cu, ws, k, &ci)) return;
   const int len = ci.len;
@@ -446,27 +419,52 @@ __global__ void __launch_bounds__(kGramThreads)
   float* sZ = nullptr;   // the heads' entering states, [8][NR] (bf16) or rows 64..71 of sB (fp32)
   float* sB = nullptr;
   float* sC = nullptr;
+  float* sW = nullptr;  // (pass 1) after the staged rows
   __nv_bfloat16* sBh = nullptr;
   __nv_bfloat16* sCh = nullptr;
   const int NSh = gram_stride_h(N);
   if constexpr (!OUT) {
-    sB = rest;
-    stage_chunk_rows<false>(sB, nullptr, NS, Bp, Bp, row0, rstride, len, N, NR, vec, tid);
-  } else {
-    sG = rest;
-    sCz = sG + kDenQ * (kDenQ + 1);
-    float* after = sCz + kDenQ * kDenHeads;
     if constexpr (kH) {
-      sZ = after;  // [8][NS]
-      sBh = reinterpret_cast<__nv_bfloat16*>(sZ + kDenHeads * NS);
-      sCh = sBh + kDenQ * NSh;
-      stage_chunk_rows_h(sBh, sCh, NSh, reinterpret_cast<const __nv_bfloat16*>(B),
-                         reinterpret_cast<const __nv_bfloat16*>(C), row0, rstride, len, N, NR, vec, tid);
-      for (int i = tid; i < kDenHeads * NR; i += kGramThreads) {
-        const int hh = i / NR, n = i % NR;
-        sZ[hh * NS + n] = (hh < nh && n < N) ? ws.states[(k * g.H + h0 + hh) * (int64_t)N + n] : 0.f;
-      }
+      sBh = reinterpret_cast<__nv_bfloat16*>(rest);
+      sW = reinterpret_cast<float*>(sBh + kDenQ * NSh);
+      stage_rows_h(sBh, NSh, reinterpret_cast<const __nv_bfloat16*>(B), row0, rstride, len, N, NR, vec, tid);
+      cp_async_wait_all();
     } else {
+      sB = rest;
+      sW = sB + kDenQ * NS;
+      stage_chunk_rows<false>(sB, nullptr, NS, Bp, Bp, row0, rstride, len, N, NR, vec, tid);
+    }
+  } else {
+    if constexpr (kH) {
+      // sZ [8][NS], then the B rows (G over them once read), then the C rows (<C, z_in> over them)
+      sZ = rest;
+      sBh = reinterpret_cast<__nv_bfloat16*>(sZ + kDenHeads * NS);
+      sCh = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<unsigned char*>(sBh) + den_gram_rows_h(N));
+      sG = reinterpret_cast<float*>(sBh);
+      sCz = reinterpret_cast<float*>(sCh);
+      stage_rows_h(sBh, NSh, reinterpret_cast<const __nv_bfloat16*>(B), row0, rstride, len, N, NR, vec, tid);
+      stage_rows_h(sCh, NSh, reinterpret_cast<const __nv_bfloat16*>(C), row0, rstride, len, N, NR, vec, tid);
+      if (vec) {
+        // the entering states, 4 floats per copy (N is a multiple of 8 here)
+        const int zpr = NR / 4;
+        const uint32_t z0 = static_cast<uint32_t>(__cvta_generic_to_shared(sZ));
+        for (int i = tid; i < kDenHeads * zpr; i += kGramThreads) {
+          const int hh = i / zpr, c = (i % zpr) * 4;
+          const bool ok = hh < nh && c < N;
+          cp_async16(z0 + (uint32_t)((hh * NS + c) * 4),
+                     ok ? ws.states + (k * g.H + h0 + hh) * (int64_t)N + c : ws.states, ok ? 16 : 0);
+        }
+      } else {
+        for (int i = tid; i < kDenHeads * NR; i += kGramThreads) {
+          const int hh = i / NR, n = i % NR;
+          sZ[hh * NS + n] = (hh < nh && n < N) ? ws.states[(k * g.H + h0 + hh) * (int64_t)N + n] : 0.f;
+        }
+      }
+      cp_async_wait_all();
+    } else {
+      sG = rest;
+      sCz = sG + kDenQ * (kDenQ + 1);
+      float* after = sCz + kDenQ * kDenHeads;
       sB = after;                          // [64 + 8][NS]: B rows, then the entering states
       sC = sB + (kDenQ + kDenHeads) * NS;  // [64][NS]
       sZ = sB + kDenQ * NS;
@@ -489,14 +487,23 @@ __global__ void __launch_bounds__(kGramThreads)
       if (lane >= o) c0 += u0, c1 += u1;
     }
     c1 += __shfl_sync(0xffffffffu, c0, 31);
-    sdl[w * kDenQ + lane] = d0;
-    sdl[w * kDenQ + lane + 32] = d1;
+    if constexpr (OUT) {
+      // log2 units: scs = cs log2 e for the token side, sdl = cs log2 e - log2 delta for the
+      // source side (+inf past the chunk's tokens), so a decay weight is ex2(scs_t - sdl_s)
+      c0 *= kLog2e;
+      c1 *= kLog2e;
+      sdl[w * kDenQ + lane] = c0 - log2f(d0);
+      sdl[w * kDenQ + lane + 32] = c1 - log2f(d1);
+    } else {
+      sdl[w * kDenQ + lane] = d0;
+      sdl[w * kDenQ + lane + 32] = d1;
+    }
     scs[w * kDenQ + lane] = c0;
     scs[w * kDenQ + lane + 32] = c1;
   }
   __syncthreads();
   if constexpr (!OUT) {
-    float* sw = sB + kDenQ * NS;          // [8][64] weights exp(cs_last - cs_s) delta_s
+    float* sw = sW;                       // [8][64] weights exp(cs_last - cs_s) delta_s
     float* red = sw + kDenHeads * kDenQ;  // [8][parts * N] partial sums
     for (int i = tid; i < kDenHeads * kDenQ; i += kGramThreads) {
       const int hh = i / kDenQ;
@@ -510,7 +517,11 @@ __global__ void __launch_bounds__(kGramThreads)
 #pragma unroll
       for (int hh = 0; hh < kDenHeads; ++hh) acc[hh] = 0.f;
       for (int t = part; t < len; t += parts) {
-        const float bv = sB[t * NS + n];
+        float bv;
+        if constexpr (kH)
+          bv = __bfloat162float(sBh[t * NSh + n]);
+        else
+          bv = sB[t * NS + n];
 #pragma unroll
         for (int hh = 0; hh < kDenHeads; ++hh) acc[hh] = fmaf(sw[hh * kDenQ + t], bv, acc[hh]);
       }
@@ -528,9 +539,11 @@ __global__ void __launch_bounds__(kGramThreads)
   } else {
     if constexpr (kH) {
       // G on the tensor cores: warp w computes rows 16 (w / 2).. and columns 32 (w % 2)..
-      // as four m16n8k16 tiles per 16-wide step of the state dimension
+      // as four m16n8k16 tiles per 16-wide step of the state dimension.  The even warps also
+      // take <C_t, z_in> of their 16 rows for the 8 heads, z split into bf16 hi + lo.
       const int t0 = (w >> 1) * 16, s0 = (w & 1) * 32;
-      float acc[4][4];
+      const bool cz = (w & 1) == 0;
+      float acc[4][4], czacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -548,7 +561,23 @@ __global__ void __launch_bounds__(kGramThreads)
           mma_bf16_16816(acc[2 * jp], a0, a1, a2, a3, b0, b1);
           mma_bf16_16816(acc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
         }
+        if (cz) {
+          // B fragment of z: head lane / 4, state elements kk + 2 (lane % 4) + {0, 1} (+ 8)
+          const float* zr = sZ + (lane >> 2) * NS + kk + 2 * (lane & 3);
+          const float2 zlo = *reinterpret_cast<const float2*>(zr);
+          const float2 zhi = *reinterpret_cast<const float2*>(zr + 8);
+          const __nv_bfloat162 h0v = __floats2bfloat162_rn(zlo.x, zlo.y);
+          const __nv_bfloat162 h1v = __floats2bfloat162_rn(zhi.x, zhi.y);
+          const float2 r0 = __bfloat1622float2(h0v), r1 = __bfloat1622float2(h1v);
+          const __nv_bfloat162 l0v = __floats2bfloat162_rn(zlo.x - r0.x, zlo.y - r0.y);
+          const __nv_bfloat162 l1v = __floats2bfloat162_rn(zhi.x - r1.x, zhi.y - r1.y);
+          mma_bf16_16816(czacc, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(&h0v),
+                         *reinterpret_cast<const uint32_t*>(&h1v));
+          mma_bf16_16816(czacc, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(&l0v),
+                         *reinterpret_cast<const uint32_t*>(&l1v));
+        }
       }
+      __syncthreads();  // every warp has read the B and C rows that G and <C, z_in> replace
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int sc = s0 + 8 * j + 2 * (lane & 3), t = t0 + (lane >> 2);
@@ -557,30 +586,13 @@ __global__ void __launch_bounds__(kGramThreads)
         sG[sc * (kDenQ + 1) + t + 8] = acc[j][2];
         sG[(sc + 1) * (kDenQ + 1) + t + 8] = acc[j][3];
       }
-      // <C_t, z_in> of the block's heads, thread (t, pair of heads)
-      const int t = tid >> 2, hp = (tid & 3) * 2;
-      float c0 = 0.f, c1 = 0.f;
-      for (int n = 0; n < NR; n += 8) {
-        const uint4 q = *reinterpret_cast<const uint4*>(sCh + t * NSh + n);
-        const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&q);
-        float cv[8];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const float2 f = __bfloat1622float2(q2[m]);
-          cv[2 * m] = f.x;
-          cv[2 * m + 1] = f.y;
-        }
-        const float4 za = *reinterpret_cast<const float4*>(sZ + hp * NS + n);
-        const float4 zb = *reinterpret_cast<const float4*>(sZ + hp * NS + n + 4);
-        const float4 ya = *reinterpret_cast<const float4*>(sZ + (hp + 1) * NS + n);
-        const float4 yb = *reinterpret_cast<const float4*>(sZ + (hp + 1) * NS + n + 4);
-        c0 = fmaf(cv[0], za.x, fmaf(cv[1], za.y, fmaf(cv[2], za.z, fmaf(cv[3], za.w, c0))));
-        c0 = fmaf(cv[4], zb.x, fmaf(cv[5], zb.y, fmaf(cv[6], zb.z, fmaf(cv[7], zb.w, c0))));
-        c1 = fmaf(cv[0], ya.x, fmaf(cv[1], ya.y, fmaf(cv[2], ya.z, fmaf(cv[3], ya.w, c1))));
-        c1 = fmaf(cv[4], yb.x, fmaf(cv[5], yb.y, fmaf(cv[6], yb.z, fmaf(cv[7], yb.w, c1))));
+      if (cz) {
+        const int t = t0 + (lane >> 2), hc = 2 * (lane & 3);
+        sCz[t * kDenHeads + hc] = czacc[0];
+        sCz[t * kDenHeads + hc + 1] = czacc[1];
+        sCz[(t + 8) * kDenHeads + hc] = czacc[2];
+        sCz[(t + 8) * kDenHeads + hc + 1] = czacc[3];
       }
-      sCz[t * kDenHeads + hp] = c0;
-      sCz[t * kDenHeads + hp + 1] = c1;
     } else {
       // G[t][s] for t = ti + 16 a, s = si + 16 b: with NS = 4 (mod 32) the 16 B rows a warp
       // reads land in distinct bank quads two by two (two wavefronts per float4 read)
@@ -625,26 +637,26 @@ __global__ void __launch_bounds__(kGramThreads)
     }
     __syncthreads();
     if (w < nh) {
-      // lane l: tokens l and l + 32 (delta is zero past the chunk's tokens).  A source in the
-      // first 32-block reaches token l + 32 through the block boundary:
-      // exp(cs_t - cs_s) = exp(cs_t - cs_31) exp(cs_31 - cs_s), both factors at most 1.
-      const float* dl = sdl + w * kDenQ;
+      // lane l: tokens l and l + 32.  A source in the first 32-block reaches token l + 32
+      // through the block boundary: exp(cs_t - cs_s) = exp(cs_t - cs_31) exp(cs_31 - cs_s),
+      // both factors at most 1.  In log2 units the weight of source s at token t is
+      // ex2(scs_t - sdl_s) = exp(cs_t - cs_s) delta_s.
+      const float* sv = sdl + w * kDenQ;
       const float* cs = scs + w * kDenQ;
       const float c0 = cs[lane], c1 = cs[lane + 32], cm = cs[31];
-      const float u = ex2a((cm - c0) * kLog2e) * dl[lane];
+      const float u = ex2a(cm - sv[lane]);
       float s0 = 0.f, s1 = 0.f;
       for (int sidx = 0; sidx < 32; ++sidx) {
         const float* gs = sG + sidx * (kDenQ + 1);
         const float us = __shfl_sync(0xffffffffu, u, sidx);
-        if (sidx <= lane) s0 = fmaf(ex2a((c0 - cs[sidx]) * kLog2e) * dl[sidx], gs[lane], s0);
+        if (sidx <= lane) s0 = fmaf(ex2a(c0 - sv[sidx]), gs[lane], s0);
         s1 = fmaf(us, gs[lane + 32], s1);
       }
-      s1 *= ex2a((c1 - cm) * kLog2e);
+      s1 *= ex2a(c1 - cm);
       for (int sidx = 32; sidx < kDenQ; ++sidx)
-        if (sidx <= lane + 32)
-          s1 = fmaf(ex2a((c1 - cs[sidx]) * kLog2e) * dl[sidx], sG[sidx * (kDenQ + 1) + lane + 32], s1);
-      s0 = fmaf(ex2a(c0 * kLog2e), sCz[lane * kDenHeads + w], s0);
-      s1 = fmaf(ex2a(c1 * kLog2e), sCz[(lane + 32) * kDenHeads + w], s1);
+        if (sidx <= lane + 32) s1 = fmaf(ex2a(c1 - sv[sidx]), sG[sidx * (kDenQ + 1) + lane + 32], s1);
+      s0 = fmaf(ex2a(c0), sCz[lane * kDenHeads + w], s0);
+      s1 = fmaf(ex2a(c1), sCz[(lane + 32) * kDenHeads + w], s1);
       if (lane < len) den[(ci.start + lane) * g.H + h] = s0;
       if (lane + 32 < len) den[(ci.start + lane + 32) * g.H + h] = s1;
     }
@@ -652,7 +664,7 @@ __global__ void __launch_bounds__(kGramThreads)
 }
 
 // (2): per (document, head, state element), the chunks' end states become entering
-// states; eight chunks of loads are issued ahead of their dependent updates
+// states; sixteen chunks of loads are issued ahead of their dependent updates
 __global__ void __launch_bounds__(256) den_pass_kernel(Geom g, SimtWorkspace ws) {
   const int d = blockIdx.x, h = blockIdx.y;
   const int n = blockIdx.z * 256 + threadIdx.x;
@@ -661,7 +673,7 @@ __global__ void __launch_bounds__(256) den_pass_kernel(Geom g, SimtWorkspace ws)
   int64_t first;
   const int64_t cnt = doc_chunks(g, ws, d, &first);
   float carry = 0.f;
-  constexpr int kU = 8;
+  constexpr int kU = 16;
   int64_t c = 0;
   for (; c + kU <= cnt; c += kU) {
     float s[kU], ld[kU];
