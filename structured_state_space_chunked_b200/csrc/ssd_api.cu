@@ -363,6 +363,18 @@ int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* 
   const int bf = d.in_dtype == SSD_BF16;
   const int64_t rows = tokens * d.ngroups;
   cudaError_t e = ssd::fmap_apply(feature_map, rows, (int)d.dstate, N2, bf, B, B2, C, C2, stream);
+  // Two ways to normalise.  When the numerator kernel leaves at least a quarter of the SMs
+  // idle (fewer units than 3/4 of the SMs), the denominator runs beside it on the second
+  // stream and a last pass divides y.  Otherwise the denominator runs first and the
+  // numerator kernel divides in its output epilogue, which saves the pass over y.
+  if (normalize && path == SSD_PATH_TC && ssd::tc_den_supported(g, tc_opts(h)) &&
+      4 * (int64_t)ssd::tc_units(g) > 3 * (int64_t)h->num_sms) {
+    if (e == cudaSuccess) e = ssd::den_scan(gd, cu_seqlens, dws, h->status, dt, A, dt_bias, B2, C2, den, stream);
+    ssd::Args a{x, dt, A, B2, C2, D, dt_bias, nullptr, cu_seqlens, y, final_states};
+    if (e == cudaSuccess) e = ssd::tc_forward_den(g, a, den, h->status, stream, h->num_sms, tc_opts(h));
+    if (cur != h->device) cudaSetDevice(cur);
+    return cuda_rc(e);
+  }
   if (normalize && e == cudaSuccess && !h->side) {
     e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);

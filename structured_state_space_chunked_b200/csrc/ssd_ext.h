@@ -23,6 +23,13 @@ bool den_scan_supported(int N);
 cudaError_t den_scan(const Geom& g, const int32_t* cu, void* workspace, int* status, const void* dt,
                      const float* A, const float* dt_bias, const void* B, const void* C, float* den,
                      cudaStream_t stream);
+// The tensor-core forward (ssd_tc.cu, N <= 128, 64-column units) with the division folded
+// in: y = num / den + a.D x for a denominator den [tokens][H] computed beforehand.  The
+// skip term enters the tile's mask diagonal as D den and each output row is scaled by
+// 1 / den.  tc_den_supported says whether the shape and options take that kernel.
+bool tc_den_supported(const Geom& g, const TcOpts& opts);
+cudaError_t tc_forward_den(const Geom& g, const Args& a, const float* den, int* status, cudaStream_t stream,
+                           int num_sms, const TcOpts& opts);
 // the chunk table of packed documents (the CUDA-core forward's first kernel)
 cudaError_t simt_varlen_table(const Geom& g, const int32_t* cu, const SimtWorkspace& ws, int* status,
                               cudaStream_t stream);

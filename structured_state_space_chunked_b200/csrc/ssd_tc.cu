@@ -39,6 +39,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ssd_ext.h"
 #include "ssd_internal.h"
 #include "tc_common.cuh"
 
@@ -97,6 +98,7 @@ struct KParams {
   const void* dt;
   const float* A;
   const float* D;
+  const float* den;  // optional [tokens][H]: y = num / den + D x (see tc_forward_den)
   const float* dt_bias;
   const float* init;
   const int32_t* cu;
@@ -308,7 +310,8 @@ __device__ __noinline__ int prev_unit_with_tiles(const KParams& kp, int u) {
   return -1;
 }
 
-template <int NT>
+// DEN: the division by a denominator folded in (kp.den set); the plain forward is DEN = false
+template <int NT, bool DEN = false>
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_tc_fused(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                  const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ KParams kp) {
@@ -531,10 +534,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     struct Pre {
       uint32_t dt;  // raw bf16 bits: converted only in E1, so the load latency stays hidden
-      float A, bias, D;
+      float A, bias, D, den;
     };
     auto prefetch = [&](const Cursor& c) -> Pre {
-      Pre p{0u, 0.f, 0.f, 0.f};
+      Pre p{0u, 0.f, 0.f, 0.f, 1.f};
       if (!c.valid) return p;
       const int len = min(kTile, c.U.len - c.jt * kTile);
       if (r < len)
@@ -543,6 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       p.A = kp.A[c.U.h];
       p.bias = kp.dt_bias ? kp.dt_bias[c.U.h] : 0.f;
       p.D = kp.D ? kp.D[c.U.h] : 0.f;
+      if (DEN && r < len) p.den = kp.den[(c.U.start + (int64_t)c.jt * kTile + r) * g.H + c.U.h];
       return p;
     };
 
@@ -555,7 +559,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // E1 of a tile: delta, in-tile cumulative log decay (log2 units), the per-column
     // factor v (shared through smem), the input weight w and exp(cs) for the output.
-    float cs = 0.f, dl = 0.f, wr = 0.f, el = 0.f, e0 = 0.f, e1 = 0.f, e2 = 0.f, e3 = 0.f, Dh = 0.f;
+    // With a denominator the row's skip term is D den (on the mask diagonal) and the whole
+    // output row is scaled by rs = 1 / den, so y = num / den + D x; without one both
+    // factors are exactly 1.
+    float cs = 0.f, dl = 0.f, wr = 0.f, el = 0.f, e0 = 0.f, e1 = 0.f, e2 = 0.f, e3 = 0.f, Dh = 0.f, rs = 1.f;
     auto stage1 = [&](const Cursor& c, const Pre& p) {
       const int len = min(kTile, c.U.len - c.jt * kTile);
       float la = 0.f;
@@ -582,7 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       vw[r] = ex2(cs_end - cs) * dl;
       wr = ex2(e3 - cs) * dl;  // exp(cs_last - cs) delta
       el = ex2(cs);            // exp(cs)
-      Dh = p.D;
+      Dh = DEN ? p.D * p.den : p.D;
+      rs = DEN ? 1.f / p.den : 1.f;
       sync_g();
     };
 
@@ -685,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(PREP0 + w));
 
       // ---- E1 of this group's next tile, while the tensor cores finish this one ----
-      const float el_cur = el;
+      const float el_cur = el, rs_cur = rs;
       if (nxt.valid) stage1(nxt, pn);
 
       // ---- E5: y = exp(cs) Yoff + Ydiag, staged in smem, coalesced stores ----
@@ -698,13 +706,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_ld32(yaddr + 32 * half, yo);
         tc_ld32(zaddr + 64 + 32 * half, yd);
         tc_wait_ld();
+        float yv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) yv[j] = DEN ? fmaf(el_cur, yo[j], yd[j]) * rs_cur : fmaf(el_cur, yo[j], yd[j]);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           st_shared_v4(xw_base + swz((uint32_t)r, (uint32_t)(4 * half + c)),
-                       pack_bf16(fmaf(el_cur, yo[8 * c + 0], yd[8 * c + 0]), fmaf(el_cur, yo[8 * c + 1], yd[8 * c + 1])),
-                       pack_bf16(fmaf(el_cur, yo[8 * c + 2], yd[8 * c + 2]), fmaf(el_cur, yo[8 * c + 3], yd[8 * c + 3])),
-                       pack_bf16(fmaf(el_cur, yo[8 * c + 4], yd[8 * c + 4]), fmaf(el_cur, yo[8 * c + 5], yd[8 * c + 5])),
-                       pack_bf16(fmaf(el_cur, yo[8 * c + 6], yd[8 * c + 6]), fmaf(el_cur, yo[8 * c + 7], yd[8 * c + 7])));
+                       pack_bf16(yv[8 * c + 0], yv[8 * c + 1]), pack_bf16(yv[8 * c + 2], yv[8 * c + 3]),
+                       pack_bf16(yv[8 * c + 4], yv[8 * c + 5]), pack_bf16(yv[8 * c + 6], yv[8 * c + 7]));
       }
       tc_fence_before();
       mbar_arrive(bar(Z_FREE0 + w));  // Z (mask + Ydiag) and Yoff are read: next C B^T may land
@@ -801,13 +810,10 @@ int tc_units(const Geom& g) { return g.ndocs * g.H * (g.P / kPT); }
 int tc_kernels(const Geom&) { return 1; }
 size_t tc_workspace_bytes(const Geom&) { return 256; }
 
-cudaError_t tc_forward(const Geom& g, const Args& a, void*, int* status, cudaStream_t stream,
-                       int num_sms, const TcOpts& opts) {
-  if (opts.unit_columns == 128) return tc_wide_forward(g, a, status, stream, num_sms);
-  // N > 128, and any shape whose wait bound or forced-timeout test is set: the kernel
-  // of ssd_tc2.cu (its bounded waits take the handle's limit)
-  if (tc2_supported(g) || opts.stall || opts.wait_ns != TcOpts().wait_ns)
-    return tc2_forward(g, a, status, stream, num_sms, opts.wait_ns, opts.stall);
+namespace {
+
+cudaError_t tc1_forward(const Geom& g, const Args& a, const float* den, int* status, cudaStream_t stream,
+                        int num_sms) {
   CUtensorMap tx, tb, tc;
   const cuuint64_t T = (cuuint64_t)g.tokens;
   {
@@ -828,6 +834,7 @@ cudaError_t tc_forward(const Geom& g, const Args& a, void*, int* status, cudaStr
   kp.dt = a.dt;
   kp.A = a.A;
   kp.D = a.D;
+  kp.den = den;
   kp.dt_bias = a.dt_bias;
   kp.init = a.init;
   kp.cu = a.cu;
@@ -837,7 +844,13 @@ cudaError_t tc_forward(const Geom& g, const Args& a, void*, int* status, cudaStr
   kp.pslices = g.P / kPT;
   kp.units = tc_units(g);
   const int grid = kp.units < num_sms ? kp.units : num_sms;
-  if (g.N <= 128) {
+  if (den) {
+    if (g.N > 128) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(ssd_tc_fused<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg<1>::SMEM);
+    if (e != cudaSuccess) return e;
+    ssd_tc_fused<1, true><<<grid, kThreads, Cfg<1>::SMEM, stream>>>(tx, tb, tc, kp);
+  } else if (g.N <= 128) {
     cudaError_t e = cudaFuncSetAttribute(ssd_tc_fused<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg<1>::SMEM);
     if (e != cudaSuccess) return e;
@@ -849,6 +862,29 @@ cudaError_t tc_forward(const Geom& g, const Args& a, void*, int* status, cudaStr
     ssd_tc_fused<2><<<grid, kThreads, Cfg<2>::SMEM, stream>>>(tx, tb, tc, kp);
   }
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t tc_forward(const Geom& g, const Args& a, void*, int* status, cudaStream_t stream,
+                       int num_sms, const TcOpts& opts) {
+  if (opts.unit_columns == 128) return tc_wide_forward(g, a, status, stream, num_sms);
+  // N > 128, and any shape whose wait bound or forced-timeout test is set: the kernel
+  // of ssd_tc2.cu (its bounded waits take the handle's limit)
+  if (tc2_supported(g) || opts.stall || opts.wait_ns != TcOpts().wait_ns)
+    return tc2_forward(g, a, status, stream, num_sms, opts.wait_ns, opts.stall);
+  return tc1_forward(g, a, nullptr, status, stream, num_sms);
+}
+
+bool tc_den_supported(const Geom& g, const TcOpts& opts) {
+  return opts.unit_columns == 64 && !tc2_supported(g) && !opts.stall && opts.wait_ns == TcOpts().wait_ns &&
+         g.N <= 128;
+}
+
+cudaError_t tc_forward_den(const Geom& g, const Args& a, const float* den, int* status, cudaStream_t stream,
+                           int num_sms, const TcOpts& opts) {
+  if (!den || !tc_den_supported(g, opts)) return cudaErrorInvalidValue;
+  return tc1_forward(g, a, den, status, stream, num_sms);
 }
 
 }  // namespace ssd
