@@ -349,6 +349,22 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
                : "r"(addr));
 }
 
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// a pair of fp32 values as bf16 hi and lo halves (about 16 significant bits together)
+__device__ __forceinline__ void split_pair(float2 v, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  const float2 r = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(v.x - r.x, v.y - r.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -510,6 +526,37 @@ __global__ void __launch_bounds__(kGramThreads)
       sw[i] = hh < nh ? expf(scs[hh * kDenQ + kDenQ - 1] - scs[i]) * sdl[i] : 0.f;
     }
     __syncthreads();
+    if constexpr (kH) {
+      // z_end = B^T W on the tensor cores: warp w takes the 16-row blocks w, w + 8, ... of
+      // the state dimension; A = B^T from the staged rows by transposing loads, W (tokens x
+      // heads) as bf16 hi + lo
+      const uint32_t aB = static_cast<uint32_t>(__cvta_generic_to_shared(sBh));
+      for (int mb = w; mb < NR / 16; mb += 8) {
+        float zacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < kDenQ; kk += 16) {
+          uint32_t a0, a1, a2, a3, bh0, bl0, bh1, bl1;
+          const int t = kk + (lane & 7) + ((lane >> 4) << 3);
+          const int col = mb * 16 + (((lane >> 3) & 1) << 3);
+          ldsm_x4_trans(aB + (uint32_t)((t * NSh + col) * 2), a0, a1, a2, a3);
+          // B fragment of W: head lane / 4, tokens kk + 2 (lane % 4) + {0, 1} (+ 8)
+          const float* wr = sw + (lane >> 2) * kDenQ + kk + 2 * (lane & 3);
+          split_pair(*reinterpret_cast<const float2*>(wr), bh0, bl0);
+          split_pair(*reinterpret_cast<const float2*>(wr + 8), bh1, bl1);
+          mma_bf16_16816(zacc, a0, a1, a2, a3, bh0, bh1);
+          mma_bf16_16816(zacc, a0, a1, a2, a3, bl0, bl1);
+        }
+        const int n = mb * 16 + (lane >> 2), hc = 2 * (lane & 3);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int nn = n + (q >> 1) * 8, hh = hc + (q & 1);
+          if (nn < N && hh < nh) ws.states[(k * g.H + h0 + hh) * (int64_t)N + nn] = zacc[q];
+        }
+      }
+      if (tid < nh)
+        ws.cs[((int64_t)(h0 + tid) * g.nchunks_max + k) * g.Q + g.Q - 1] = scs[tid * kDenQ + kDenQ - 1];
+      return;
+    }
     // thread (part, n) sums tokens part, part + parts, ... of column n for every head
     const int parts = max(1, kGramThreads / N), n = tid % N, part = tid / N;
     if (part < parts) {
@@ -517,11 +564,7 @@ __global__ void __launch_bounds__(kGramThreads)
 #pragma unroll
       for (int hh = 0; hh < kDenHeads; ++hh) acc[hh] = 0.f;
       for (int t = part; t < len; t += parts) {
-        float bv;
-        if constexpr (kH)
-          bv = __bfloat162float(sBh[t * NSh + n]);
-        else
-          bv = sB[t * NS + n];
+        const float bv = sB[t * NS + n];
 #pragma unroll
         for (int hh = 0; hh < kDenHeads; ++hh) acc[hh] = fmaf(sw[hh * kDenQ + t], bv, acc[hh]);
       }
@@ -564,17 +607,11 @@ __global__ void __launch_bounds__(kGramThreads)
         if (cz) {
           // B fragment of z: head lane / 4, state elements kk + 2 (lane % 4) + {0, 1} (+ 8)
           const float* zr = sZ + (lane >> 2) * NS + kk + 2 * (lane & 3);
-          const float2 zlo = *reinterpret_cast<const float2*>(zr);
-          const float2 zhi = *reinterpret_cast<const float2*>(zr + 8);
-          const __nv_bfloat162 h0v = __floats2bfloat162_rn(zlo.x, zlo.y);
-          const __nv_bfloat162 h1v = __floats2bfloat162_rn(zhi.x, zhi.y);
-          const float2 r0 = __bfloat1622float2(h0v), r1 = __bfloat1622float2(h1v);
-          const __nv_bfloat162 l0v = __floats2bfloat162_rn(zlo.x - r0.x, zlo.y - r0.y);
-          const __nv_bfloat162 l1v = __floats2bfloat162_rn(zhi.x - r1.x, zhi.y - r1.y);
-          mma_bf16_16816(czacc, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(&h0v),
-                         *reinterpret_cast<const uint32_t*>(&h1v));
-          mma_bf16_16816(czacc, a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(&l0v),
-                         *reinterpret_cast<const uint32_t*>(&l1v));
+          uint32_t zh0, zl0, zh1, zl1;
+          split_pair(*reinterpret_cast<const float2*>(zr), zh0, zl0);
+          split_pair(*reinterpret_cast<const float2*>(zr + 8), zh1, zl1);
+          mma_bf16_16816(czacc, a0, a1, a2, a3, zh0, zh1);
+          mma_bf16_16816(czacc, a0, a1, a2, a3, zl0, zl1);
         }
       }
       __syncthreads();  // every warp has read the B and C rows that G and <C, z_in> replace
