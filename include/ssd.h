@@ -283,9 +283,18 @@ SSD_API int ssd_feature_map_dim(int kind, int dstate);
  *   final_states [docs, H, N', P] fp32 or NULL: the numerator's final states;
  *   normalize 0 or 1.
  * The mapped B and C and the denominator live in the handle's workspace.  The
- * denominator runs as its own single-column scan (one warp per document and head)
- * and takes N' up to 1024.  Errors as for ssd_forward; SSD_ERR_INVALID_ARG for an
- * unknown map, SSD_ERR_UNSUPPORTED for a normalised N' over 1024.
+ * denominator is its own single-column scan in 64-token chunks and takes N' up to
+ * 1024.  With normalisation the call takes one of two orders:
+ *   - the denominator on a second CUDA stream that the handle creates on first use
+ *     (non-blocking, destroyed by ssd_destroy), forked from `stream` after the feature
+ *     maps and joined back into it before the division, so every result is still
+ *     ordered on `stream` (a graph captured from `stream` takes both branches); used
+ *     when the numerator leaves at least a quarter of the SMs idle;
+ *   - otherwise everything on `stream`: the denominator first, then the numerator
+ *     kernel with the division in its epilogue (tensor-core path, N' <= 128).
+ * Calls on one handle must not overlap (they share the workspace and the second
+ * stream).  Errors as for ssd_forward; SSD_ERR_INVALID_ARG for an unknown map,
+ * SSD_ERR_UNSUPPORTED for a normalised N' over 1024.
  */
 SSD_API int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* A,
                             const void* B, const void* C, const float* D, const float* dt_bias,
