@@ -376,9 +376,21 @@ int ssd_forward_ext(ssd_handle_t h, const void* x, const void* dt, const float* 
     return cuda_rc(e);
   }
   if (normalize && e == cudaSuccess && !h->side) {
-    e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
+    // all three or none, so a failed creation leaves the handle as it was
+    cudaStream_t sd = nullptr;
+    cudaEvent_t ef = nullptr, ejn = nullptr;
+    e = cudaStreamCreateWithFlags(&sd, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ef, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ejn, cudaEventDisableTiming);
+    if (e == cudaSuccess) {
+      h->side = sd;
+      h->ev_fork = ef;
+      h->ev_join = ejn;
+    } else {
+      if (ejn) cudaEventDestroy(ejn);
+      if (ef) cudaEventDestroy(ef);
+      if (sd) cudaStreamDestroy(sd);
+    }
   }
   if (normalize && e == cudaSuccess) e = cudaEventRecord(h->ev_fork, stream);
   // the numerator (D added after the division when normalising)
