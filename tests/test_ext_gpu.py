@@ -42,6 +42,9 @@ CASES = [
     ("bf16", 2, 700, 24, 64, 128, 1, ssd.SSD_FMAP_RELU, True, 0, 256),
     ("bf16", 1, 0, 24, 64, 64, 2, ssd.SSD_FMAP_RELU, True, 1300, 256),
     ("fp32", 1, 300, 3, 16, 16, 1, ssd.SSD_FMAP_REBASED, True, 0, 64),
+    # bf16 with a mapped dstate that is no multiple of 8 (Based, N = 8 -> 73): the
+    # denominator's element-by-element staging and its products over zero-padded columns
+    ("bf16", 2, 300, 8, 64, 8, 1, ssd.SSD_FMAP_BASED, True, 0, 64),
     # 128 or more tensor-core units (more than 3/4 of a B200's 148 SMs): the denominator
     # first, the division folded into the numerator kernel's output epilogue
     ("bf16", 2, 700, 64, 64, 128, 1, ssd.SSD_FMAP_RELU, True, 0, 256),
@@ -51,7 +54,7 @@ IDS = ["silu-simt", "relu-norm-simt", "based-norm-simt-fp32", "rebased-norm-simt
        "based-norm-packed-simt", "none-norm-fp32", "relu-fp32",
        "silu-tc", "relu-norm-tc", "rebased-norm-tc", "rebased-norm-packed-tc",
        "relu-norm-tc-h24", "relu-norm-packed-tc-hpg12", "rebased-norm-fp32-n256",
-       "relu-norm-tc-folded", "relu-norm-packed-tc-folded"]
+       "based-norm-bf16-n73", "relu-norm-tc-folded", "relu-norm-packed-tc-folded"]
 
 
 @pytest.mark.parametrize("case", CASES, ids=IDS)
